@@ -1,0 +1,454 @@
+"""Benchmark of the chunked-SGMV LoRA shrink/expand pair on B200.
+
+Workload: the Qwen3-8B-like q/k/v decode case -- K=4096, three output slices
+of 4096/1024/1024 columns, 8 adapters of rank 16 in bf16, one segment per
+adapter, shuffled permutation -- swept over tok = 50 ... 8192.  One step is
+one pass of the hot path over the sweep: for every tok, lora_shrink and then
+lora_expand of the shrink's own output (18 calls).  The L2 cache is flushed
+(256 MB write) before every call and each call is bracketed by CUDA events on
+the launching stream, as on the sgl-kernel-xpu page ("Performance":
+do_bench with the L2 flushed between runs).
+
+value = algorithmic bytes of all calls / their summed device time (GB/s),
+with bytes = gathered x + A of the adapters used + rank activations written
+(shrink) and rank activations + B + base read and written (expand).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs the same sweep on its own GPU (independent
+batches, no collective on the data path: weak scaling); rank 0 prints one JSON
+line with the whole-job value (sum over ranks / max-over-ranks time).
+"""
+import argparse
+import hashlib
+import glob
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from scatter_gemm_b200 import workloads as W  # noqa: E402
+
+METRIC = "LoRA shrink/expand effective GB/s (bf16, tok 50–8192) and % of HBM peak"
+WORKLOAD = ("qkv decode sweep: K=4096, slices q/k/v 4096/1024/1024, 8 adapters rank 16 bf16, "
+            "one segment per adapter, shuffled permutation, tok 50..8192; step = shrink then "
+            "expand at every tok")
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def csrc_hash():
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "scatter_gemm_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic():
+    """ncu DRAM traffic of the dominant kernel, if taken on the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("csrc_hash") != csrc_hash():
+        return None
+    return d
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        p = torch.cuda.get_device_properties(device)
+        self.bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", self.bus],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.25)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------
+# device problem
+# ----------------------------------------------------------------------------
+
+class DevProblem:
+    def __init__(self, p, device):
+        self.p = p
+        tdt = torch.bfloat16 if p.dtype == "bf16" else torch.float16
+
+        def up(bits):
+            return torch.from_numpy(bits.view(np.int16)).to(device).view(tdt)
+
+        self.x = up(p.x)
+        self.A = up(p.A)
+        self.B = up(p.B)
+        self.base = up(p.base)
+        self.si = torch.from_numpy(p.seg_indptr).to(device)
+        self.wi = torch.from_numpy(p.weight_indices).to(device)
+        self.pm = torch.from_numpy(p.permutation).to(device)
+        self.sc = torch.from_numpy(p.scalings).to(device)
+        self.out = torch.zeros(p.tok, p.S * p.rs, dtype=tdt, device=device)
+        self.off = [int(v) for v in p.slice_offsets]
+        from scatter_gemm_b200 import lora
+        self.ws = lora.make_workspace(p.tok, p.nseg, p.L, device)
+        self.bytes_shrink = W.bytes_shrink(p)
+        self.bytes_expand = W.bytes_expand(p)
+
+    def shrink(self, lora):
+        lora.lora_shrink(self.x, self.A, self.si, self.wi, self.pm, self.out,
+                         num_slices=self.p.S, rank=self.p.r, workspace=self.ws)
+
+    def expand(self, lora):
+        lora.lora_expand(self.out, self.B, self.si, self.wi, self.pm, self.off, self.sc,
+                         self.base, rank=self.p.r, workspace=self.ws)
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (baseline; never the product path)
+# ----------------------------------------------------------------------------
+
+def time_oracle(toks, min_seconds):
+    import oracle
+    probs = [W.make_problem("qkv", seed=0, tok=t) for t in toks]
+    nbytes = sum(W.bytes_shrink(p) + W.bytes_expand(p) for p in probs)
+    t0 = time.perf_counter()
+    passes = 0
+    while True:
+        for p in probs:
+            h = oracle.shrink_problem(p)
+            oracle.expand_problem(p, in_r=h)
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    return nbytes * passes / el / 1e9, el, passes, oracle.max_threads()
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle timed on the host cores, rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+    toks = (50,)
+    probs = [W.make_problem("qkv", seed=0, tok=t) for t in toks]
+    nbytes = sum(W.bytes_shrink(p) + W.bytes_expand(p) for p in probs)
+
+    def step():
+        for p in probs:
+            h = oracle.shrink_problem(p)
+            oracle.expand_problem(p, in_r=h)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = nbytes * args.steps / el / 1e9
+    cores = oracle.max_threads()
+    sample = ("one shrink + expand of the tok=50 case of the sweep per step "
+              "(CPU oracle, fp32 sequential sums)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def run_ours(args, rank, world, device):
+    from scatter_gemm_b200 import lora
+    import torch.distributed as dist
+
+    toks = [int(t) for t in args.toks.split(",")]
+    probs = [DevProblem(W.make_problem("qkv", seed=rank, tok=t), device) for t in toks]
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream()
+    n_calls = 2 * len(probs)
+
+    def step(ev):
+        for j, dp in enumerate(probs):
+            flush.zero_()
+            if ev is not None:
+                ev[2 * j][0].record(stream)
+            dp.shrink(lora)
+            if ev is not None:
+                ev[2 * j][1].record(stream)
+            flush.zero_()
+            if ev is not None:
+                ev[2 * j + 1][0].record(stream)
+            dp.expand(lora)
+            if ev is not None:
+                ev[2 * j + 1][1].record(stream)
+
+    for _ in range(args.warmup):
+        step(None)
+    torch.cuda.synchronize()
+
+    events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n_calls)] for _ in range(args.steps)]
+    wall0, wall1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(device) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+    lora.reset_launch_count()
+    wall0.record(stream)
+    for k in range(args.steps):
+        step(events[k])
+    wall1.record(stream)
+    torch.cuda.synchronize()
+    launches = lora.launch_count()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if clocks else None
+
+    # per-call device times (ms), [steps, calls]
+    t = np.array([[s.elapsed_time(e) for (s, e) in row] for row in events], dtype=np.float64)
+    kernel_ms = float(t.sum())
+    wall_ms = wall0.elapsed_time(wall1)
+    bytes_step = sum(dp.bytes_shrink + dp.bytes_expand for dp in probs)
+    if world > 1:
+        red = torch.tensor([kernel_ms, wall_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(red, op=dist.ReduceOp.MAX)
+        kernel_ms, wall_ms = float(red[0]), float(red[1])
+
+    # e2e: host buffers in pinned memory, H2D + both calls + D2H inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, probs, lora, device, stream, world)
+
+    if rank != 0:
+        return
+    peak, peak_kind = measured_peaks()
+    med = np.median(t, axis=0)  # per call, ms
+    detail = []
+    fr = []
+    for j, dp in enumerate(probs):
+        s_ms, e_ms = med[2 * j], med[2 * j + 1]
+        gbs = (dp.bytes_shrink + dp.bytes_expand) / ((s_ms + e_ms) * 1e-3) / 1e9
+        detail.append({"tok": dp.p.tok,
+                       "shrink_us": round(s_ms * 1e3, 2), "expand_us": round(e_ms * 1e3, 2),
+                       "shrink_gbs": round(dp.bytes_shrink / (s_ms * 1e-3) / 1e9, 1),
+                       "expand_gbs": round(dp.bytes_expand / (e_ms * 1e-3) / 1e9, 1),
+                       "gbs": round(gbs, 1)})
+        if dp.p.tok >= 1024:
+            fr.append(gbs)
+    geo = math.exp(sum(math.log(v) for v in fr) / len(fr)) if fr else None
+    mean_case = statistics.mean(d["gbs"] for d in detail)
+
+    # roofline of the dominant kernel (larger summed time of the two ops)
+    s_tot, e_tot = t[:, 0::2].sum(), t[:, 1::2].sum()
+    dom = "expand" if e_tot >= s_tot else "shrink"
+    cols = t[:, 1::2] if dom == "expand" else t[:, 0::2]
+    alg = [dp.bytes_expand if dom == "expand" else dp.bytes_shrink for dp in probs]
+    achieved = sum(alg) * args.steps / (cols.sum() * 1e-3) / 1e9
+    tr = load_traffic()
+    traffic = None
+    if tr is not None and tr.get("op") == dom:
+        traffic = tr.get("dram_bytes_per_launch")
+    roof = {"bound": "hbm", "kernel": f"lora_{dom} kernels over the sweep",
+            "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
+            "traffic": traffic,
+            "algorithmic_bytes_per_launch": round(sum(alg) / len(alg)),
+            "share_of_step": round(float(max(s_tot, e_tot) / (s_tot + e_tot)), 3)}
+
+    cpu = None
+    if world == 1 and not args.no_cpu:
+        v, el, passes, cores = time_oracle([50, 128, 256, 512, 1024], args.cpu_seconds)
+        cpu = {"value": round(v, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": f"tok 50,128,256,512,1024 of the sweep, shrink + expand, "
+                         f"{passes} pass(es) in {el:.1f} s"}
+
+    value = bytes_step * args.steps * world / (kernel_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(kernel_ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "toks": toks, "l2": "flushed before every call "
+                   "(256 MB write, outside the events)", "parallelism": f"dp{world}",
+                   "step_ms_incl_flush": round(wall_ms / args.steps, 4)},
+        "frac_of_peak": round(value / world / peak, 4),
+        "frac_of_nominal_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
+        "geomean_gbs_tok_ge_1024": round(geo, 1) if geo else None,
+        "geomean_frac_tok_ge_1024": round(geo / peak, 4) if geo else None,
+        "geomean_frac_nominal_tok_ge_1024": round(geo / NOMINAL_HBM_GBS, 4) if geo else None,
+        "mean_case_gbs": round(mean_case, 1),
+        "per_tok": detail,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(launches) * world,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, probs, lora, device, stream, world):
+    """Same sweep through the public API with host buffers: H2D of the step's
+    inputs (x, tables, base) from pinned memory, both calls, D2H of base."""
+    import torch.distributed as dist
+    host = []
+    for dp in probs:
+        h = {k: getattr(dp, k).cpu().pin_memory() for k in ("x", "base", "si", "wi", "pm")}
+        h["base_back"] = torch.empty_like(h["base"]).pin_memory()
+        host.append(h)
+    h2d = sum(sum(v.numel() * v.element_size() for k, v in h.items() if k != "base_back")
+              for h in host)
+    d2h = sum(h["base_back"].numel() * h["base_back"].element_size() for h in host)
+    steps = max(3, min(args.steps, args.e2e_steps))
+
+    def step():
+        for dp, h in zip(probs, host):
+            dp.x.copy_(h["x"], non_blocking=True)
+            dp.base.copy_(h["base"], non_blocking=True)
+            dp.si.copy_(h["si"], non_blocking=True)
+            dp.wi.copy_(h["wi"], non_blocking=True)
+            dp.pm.copy_(h["pm"], non_blocking=True)
+            dp.shrink(lora)
+            dp.expand(lora)
+            h["base_back"].copy_(dp.base, non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        red = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(red, op=dist.ReduceOp.MAX)
+        ms = float(red[0])
+    nbytes = sum(dp.bytes_shrink + dp.bytes_expand for dp in probs) * steps * world
+    return {"value": round(nbytes / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--toks", default=",".join(str(t) for t in W.QKV_TOK_SWEEP))
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    try:
+        run_ours(args, rank, world, device)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,169 @@
+/* lora_sgmv.h -- C ABI of liblora_sgmv, the multi-adapter LoRA chunked-SGMV
+ * shrink/expand pair for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow the sgl-kernel-xpu page "Decode LoRA kernels are
+ * optimized" (section "Summary": the shrink gathers token rows of x through a
+ * permutation and multiplies each segment by its adapter's A; the expand
+ * multiplies those rank activations by the segment's adapter B, scales the
+ * result and scatter-adds it into column slices of the base projection
+ * output; section "Behaviour changes": the tables seg_indptr, adapter index,
+ * permutation and offset table, and the contract that callers pass one
+ * coalesced segment per adapter).  The update itself is the LoRA update of
+ * the ms-swift page "Add optional fast lora path for qwen2/qwen3 on npu"
+ * (section "Compatibility checks": no dropout, one adapter per token).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Element type: bf16 or fp16 (lora_dtype), the same for every floating
+ *    tensor of a call except `scalings`, which is fp32.  Accumulation is fp32;
+ *    each output element is rounded once, to nearest even.
+ *  - All tensors are row-major with an explicit leading dimension (in
+ *    elements).  Any element-aligned pointer is accepted; faster kernels are
+ *    picked at run time when pointers and leading dimensions are 16-byte
+ *    aligned.
+ *  - Tables (int32, in device memory):
+ *      seg_indptr[nseg+1]   segment s covers sorted rows [seg_indptr[s], seg_indptr[s+1]);
+ *                           non-decreasing, inside [0, tok]; empty segments allowed;
+ *                           rows outside [seg_indptr[0], seg_indptr[nseg]) are not touched.
+ *      weight_indices[nseg] adapter of segment s, in [0, L).
+ *      permutation[tok]     sorted row i belongs to token permutation[i]; a bijection of
+ *                           [0, tok).  NULL means the identity.
+ *  - Rank layout: an adapter has S slices (q/k/v: S = 3, gate/up: S = 2) of
+ *    valid rank r stored with stride rs >= r.  Storage padding (j >= r) is
+ *    never read and never written.
+ *  - Rank activations (out_r of the shrink, in_r of the expand) are stored in
+ *    SORTED order: row i holds token permutation[i]; slice q occupies columns
+ *    [q*rs, q*rs + r).
+ *  - Nothing is synchronised with the host: the calls read no table on the
+ *    host, enqueue their kernels on `stream` (a cudaStream_t, NULL = legacy
+ *    default stream) and return.  The library allocates no device memory and
+ *    keeps no state between calls; calls are thread-safe.
+ *  - Invalid table VALUES (a decreasing seg_indptr, an adapter index out of
+ *    range, a permutation that is not a bijection) are undefined behaviour in
+ *    lora_shrink / lora_expand, as on the pages (section "Behaviour changes");
+ *    lora_validate checks them.  Every index a kernel reads is clamped to its
+ *    tensor, so bad tables give wrong values, never an out-of-bounds access.
+ *  - Errors in the ARGUMENTS (null pointers, sizes, strides, dtype) are
+ *    reported before anything is enqueued.
+ */
+#ifndef LORA_SGMV_H
+#define LORA_SGMV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LORA_API __attribute__((visibility("default")))
+#else
+#define LORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LORA_OK = 0,
+  LORA_ERR_INVALID_ARGUMENT = 1, /* null pointer, negative or inconsistent size or stride   */
+  LORA_ERR_UNSUPPORTED = 2,      /* valid but not implemented (dtype, sizes beyond limits)   */
+  LORA_ERR_CUDA = 3,             /* a CUDA runtime call or a kernel launch failed            */
+  LORA_ERR_BAD_VALUES = 4        /* lora_validate only: the tables hold invalid values       */
+} lora_status;
+
+typedef enum { LORA_BF16 = 0, LORA_FP16 = 1 } lora_dtype;
+
+/* Bits that lora_validate writes into *d_result. */
+enum {
+  LORA_BAD_INDPTR = 2,      /* seg_indptr decreasing or outside [0, tok]       */
+  LORA_BAD_ADAPTER = 4,     /* a weight index outside [0, L)                   */
+  LORA_BAD_PERMUTATION = 8, /* permutation not a bijection of [0, tok)         */
+  LORA_BAD_SLICES = 16      /* slice_offsets negative, decreasing or > ld_base */
+};
+
+/* Limits of this build. */
+#define LORA_MAX_SLICES 8
+
+/* lora_shrink -- the shrink of the chunked-SGMV pair (page section "Summary").
+ *
+ *   out_r[i, q*rs + j] = round( sum_{k<K} x[permutation[i], k] * A_stack[a, q*rs + j, k] )
+ *   for every segment s, a = weight_indices[s], i in its rows, q < S, j < r.
+ *
+ *   x        [tok, ld_x]      device, ld_x >= K; read
+ *   A_stack  [L, S*rs, K]     device, contiguous (K contiguous, "output-dim major"); read
+ *   out_r    [tok, ld_out]    device, ld_out >= S*rs; only the valid columns of rows in
+ *                             segments are written
+ *   workspace, workspace_bytes  optional device scratch (may be NULL / 0).  With at least
+ *                             lora_workspace_size(tok, nseg, L) bytes the call may group
+ *                             the rows of many small segments by adapter first; the results
+ *                             agree within rounding either way.  It must not be used by
+ *                             another call that runs at the same time.
+ * Returns LORA_OK, LORA_ERR_INVALID_ARGUMENT, LORA_ERR_UNSUPPORTED or LORA_ERR_CUDA.
+ * tok == 0 or nseg == 0 returns LORA_OK and enqueues nothing.
+ */
+LORA_API lora_status lora_shrink(const void* x, int64_t ld_x, const void* A_stack,
+                        const int32_t* seg_indptr, const int32_t* weight_indices,
+                        const int32_t* permutation, void* out_r, int64_t ld_out,
+                        int tok, int K, int S, int r, int rs, int nseg, int L,
+                        lora_dtype dtype, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* lora_expand -- the expand of the chunked-SGMV pair (page section "Summary").
+ *
+ *   for every segment s with a = weight_indices[s] and scalings[a] != 0, every row i of s,
+ *   every slice q < S and column c in [slice_offsets[q], slice_offsets[q+1]):
+ *     t = permutation[i]
+ *     base_out[t, c] = round( base_out[t, c]
+ *                            + scalings[a] * sum_{j<r} in_r[i, q*rs + j] * B_stack[a, c - off0, j] )
+ *   with off0 = slice_offsets[0].  A segment whose scaling is exactly 0 is skipped: its
+ *   base rows stay bit-identical.
+ *
+ *   in_r           [tok, ld_in]       device, ld_in >= S*rs; read (valid columns only)
+ *   B_stack        [L, N_tot, rs]     device, contiguous, N_tot = off[S] - off[0]; read
+ *   slice_offsets  [S+1]              HOST int32 array, non-decreasing, off[S] <= ld_base;
+ *                                     read during the call only (no device copy, no sync)
+ *   scalings       [L]                device fp32
+ *   base_out       [tok, ld_base]     device; read and written in place
+ *   workspace      as for lora_shrink.
+ * Returns as lora_shrink.
+ */
+LORA_API lora_status lora_expand(const void* in_r, int64_t ld_in, const void* B_stack,
+                        const int32_t* seg_indptr, const int32_t* weight_indices,
+                        const int32_t* permutation, const int32_t* slice_offsets,
+                        const float* scalings, void* base_out, int64_t ld_base,
+                        int tok, int S, int r, int rs, int nseg, int L,
+                        lora_dtype dtype, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* Bytes of optional workspace that lets lora_shrink / lora_expand use the
+ * adapter-grouped schedule for tables with many small segments. */
+LORA_API size_t lora_workspace_size(int tok, int nseg, int L);
+
+/* lora_validate -- the value checks of the tables (page section "Behaviour
+ * changes": seg_indptr, index range, permutation, offset table), run on the
+ * device.  Writes the OR of the LORA_BAD_* bits that apply into *d_result
+ * (device int32, overwritten; 0 = valid).  slice_offsets is a HOST array and
+ * may be NULL (then the offset table is not checked); it is checked on the
+ * host and its bit is folded into *d_result.  Needs device scratch of
+ * lora_validate_workspace_size(tok) bytes.  Asynchronous: read *d_result after
+ * synchronising `stream`.
+ */
+LORA_API lora_status lora_validate(const int32_t* seg_indptr, const int32_t* weight_indices,
+                          const int32_t* permutation, const int32_t* slice_offsets,
+                          int tok, int nseg, int L, int S, int64_t ld_base,
+                          int32_t* d_result, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+LORA_API size_t lora_validate_workspace_size(int tok);
+
+/* Static description of a status code; never NULL. */
+LORA_API const char* lora_status_string(lora_status status);
+
+/* Kernel launches this thread has enqueued through the library since the last
+ * reset (a host-side counter, for accounting in benchmarks). */
+LORA_API uint64_t lora_launch_count(void);
+LORA_API void lora_reset_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LORA_SGMV_H */

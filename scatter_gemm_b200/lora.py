@@ -1,0 +1,245 @@
+"""Thin ctypes binding of liblora_sgmv (argument marshalling only).
+
+Every step of the shrink and expand runs in the CUDA library; this module
+checks torch-side metadata (device, dtype, strides) on the host, takes
+``data_ptr()`` of each tensor and the current CUDA stream, and calls the C
+ABI declared in ``include/lora_sgmv.h``.  There is no fallback: if the
+library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblora_sgmv.so")
+
+LORA_OK, LORA_ERR_INVALID_ARGUMENT, LORA_ERR_UNSUPPORTED, LORA_ERR_CUDA, LORA_ERR_BAD_VALUES = \
+    range(5)
+BAD_INDPTR, BAD_ADAPTER, BAD_PERMUTATION, BAD_SLICES = 2, 4, 8, 16
+MAX_SLICES = 8
+
+_P, _I, _L, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+_lib = None
+_lock = threading.Lock()
+
+
+class LoraError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status_string(status)} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    """Loads liblora_sgmv.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with `python -m scatter_gemm_b200.build`")
+            l = ctypes.CDLL(LIB_PATH)
+            l.lora_shrink.argtypes = [_P, _L, _P, _P, _P, _P, _P, _L] + [_I] * 8 + [_P, _Z, _P]
+            l.lora_shrink.restype = _I
+            l.lora_expand.argtypes = [_P, _L, _P, _P, _P, _P, _P, _P, _P, _L] + [_I] * 7 + \
+                [_P, _Z, _P]
+            l.lora_expand.restype = _I
+            l.lora_validate.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _L, _P, _P, _Z, _P]
+            l.lora_validate.restype = _I
+            l.lora_workspace_size.argtypes = [_I, _I, _I]
+            l.lora_workspace_size.restype = _Z
+            l.lora_validate_workspace_size.argtypes = [_I]
+            l.lora_validate_workspace_size.restype = _Z
+            l.lora_status_string.argtypes = [_I]
+            l.lora_status_string.restype = ctypes.c_char_p
+            l.lora_launch_count.argtypes = []
+            l.lora_launch_count.restype = ctypes.c_uint64
+            l.lora_reset_launch_count.argtypes = []
+            l.lora_reset_launch_count.restype = None
+            _lib = l
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().lora_status_string(status).decode()
+
+
+def launch_count() -> int:
+    return int(lib().lora_launch_count())
+
+
+def reset_launch_count() -> None:
+    lib().lora_reset_launch_count()
+
+
+def workspace_size(tok: int, nseg: int, num_adapters: int) -> int:
+    return int(lib().lora_workspace_size(tok, nseg, num_adapters))
+
+
+def make_workspace(tok: int, nseg: int, num_adapters: int, device=None) -> torch.Tensor:
+    """Allocates (through torch) the optional scratch that lets the calls
+    group many small segments by adapter."""
+    n = workspace_size(tok, nseg, num_adapters)
+    return torch.empty(max(n, 1), dtype=torch.uint8, device=device or "cuda")
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return 0
+    if t.dtype == torch.float16:
+        return 1
+    raise TypeError(f"unsupported element type {t.dtype} (bf16 or fp16)")
+
+
+def _row_major(t: torch.Tensor, name: str, dims: int = 2) -> int:
+    if t.dim() != dims:
+        raise ValueError(f"{name} must be {dims}-D, got {tuple(t.shape)}")
+    if t.stride(-1) != 1:
+        raise ValueError(f"{name} must have a unit inner stride")
+    return t.stride(0) if dims == 2 else 0
+
+
+def _table(t: Optional[torch.Tensor], name: str, allow_none: bool = False):
+    if t is None:
+        if allow_none:
+            return None
+        raise ValueError(f"{name} is required")
+    if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ws(workspace: Optional[torch.Tensor]):
+    if workspace is None:
+        return None, 0
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size()
+
+
+def lora_shrink(x: torch.Tensor, A_stack: torch.Tensor, seg_indptr: torch.Tensor,
+                weight_indices: torch.Tensor, permutation: Optional[torch.Tensor],
+                out_r: torch.Tensor, *, num_slices: int, rank: Optional[int] = None,
+                workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Shrink: out_r[i, q*rs+j] = sum_k x[perm[i], k] * A_stack[a, q*rs+j, k].
+
+    x [tok, K] (unit inner stride), A_stack [L, S*rs, K] contiguous (or
+    [L, S, rs, K]), out_r [tok, >= S*rs] (unit inner stride, sorted order).
+    `rank` is the valid rank r <= rs (default rs)."""
+    dt = _dtype_code(x)
+    if A_stack.dtype != x.dtype or out_r.dtype != x.dtype:
+        raise TypeError("x, A_stack and out_r must share one element type")
+    ld_x = _row_major(x, "x")
+    ld_out = _row_major(out_r, "out_r")
+    if not A_stack.is_contiguous():
+        raise ValueError("A_stack must be contiguous")
+    S = int(num_slices)
+    if A_stack.dim() == 4:
+        L, S4, rs, K = A_stack.shape
+        if S4 != S:
+            raise ValueError("A_stack slice dimension does not match num_slices")
+    elif A_stack.dim() == 3:
+        L, srs, K = A_stack.shape
+        if srs % S:
+            raise ValueError("A_stack rows are not a multiple of num_slices")
+        rs = srs // S
+    else:
+        raise ValueError("A_stack must be [L, S*rs, K] or [L, S, rs, K]")
+    tok, Kx = x.shape
+    if Kx != K:
+        raise ValueError(f"x has K={Kx}, A_stack has K={K}")
+    r = rs if rank is None else int(rank)
+    if out_r.shape[0] != tok:
+        raise ValueError("out_r must have one row per token")
+    nseg = seg_indptr.numel() - 1
+    ws, wsb = _ws(workspace)
+    st = lib().lora_shrink(x.data_ptr(), ld_x, A_stack.data_ptr(),
+                           _table(seg_indptr, "seg_indptr"), _table(weight_indices, "weight_indices"),
+                           _table(permutation, "permutation", True), out_r.data_ptr(), ld_out,
+                           tok, K, S, r, rs, nseg, L, dt, ws, wsb, _stream(stream))
+    if st != LORA_OK:
+        raise LoraError("lora_shrink", st)
+    return out_r
+
+
+def lora_expand(in_r: torch.Tensor, B_stack: torch.Tensor, seg_indptr: torch.Tensor,
+                weight_indices: torch.Tensor, permutation: Optional[torch.Tensor],
+                slice_offsets: Sequence[int], scalings: torch.Tensor, base_out: torch.Tensor,
+                *, rank: Optional[int] = None, workspace: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+    """Expand: base_out[perm[i], c] += scalings[a] * sum_j in_r[i, q*rs+j] * B_stack[a, c-off0, j].
+
+    in_r [tok, >= S*rs] (sorted order), B_stack [L, N_tot, rs] contiguous,
+    slice_offsets: S+1 host integers, scalings [L] fp32 CUDA, base_out
+    [tok, >= off[S]] updated in place."""
+    dt = _dtype_code(base_out)
+    if in_r.dtype != base_out.dtype or B_stack.dtype != base_out.dtype:
+        raise TypeError("in_r, B_stack and base_out must share one element type")
+    if scalings.dtype != torch.float32 or not scalings.is_cuda or not scalings.is_contiguous():
+        raise ValueError("scalings must be a contiguous fp32 CUDA tensor")
+    ld_in = _row_major(in_r, "in_r")
+    ld_base = _row_major(base_out, "base_out")
+    if B_stack.dim() != 3 or not B_stack.is_contiguous():
+        raise ValueError("B_stack must be a contiguous [L, N_tot, rs] tensor")
+    L, n_tot, rs = B_stack.shape
+    off = [int(v) for v in (slice_offsets.tolist() if torch.is_tensor(slice_offsets)
+                            else slice_offsets)]
+    S = len(off) - 1
+    if S < 1 or S > MAX_SLICES:
+        raise ValueError(f"need 2..{MAX_SLICES + 1} slice offsets")
+    if off[-1] - off[0] != n_tot:
+        raise ValueError("slice_offsets span does not match B_stack rows")
+    r = rs if rank is None else int(rank)
+    tok = base_out.shape[0]
+    if in_r.shape[0] != tok:
+        raise ValueError("in_r must have one row per token")
+    nseg = seg_indptr.numel() - 1
+    off_arr = (ctypes.c_int32 * len(off))(*off)
+    ws, wsb = _ws(workspace)
+    st = lib().lora_expand(in_r.data_ptr(), ld_in, B_stack.data_ptr(),
+                           _table(seg_indptr, "seg_indptr"), _table(weight_indices, "weight_indices"),
+                           _table(permutation, "permutation", True),
+                           ctypes.cast(off_arr, ctypes.c_void_p), scalings.data_ptr(),
+                           base_out.data_ptr(), ld_base, tok, S, r, rs, nseg, L, dt, ws, wsb,
+                           _stream(stream))
+    if st != LORA_OK:
+        raise LoraError("lora_expand", st)
+    return base_out
+
+
+def lora_validate(seg_indptr: torch.Tensor, weight_indices: torch.Tensor,
+                  permutation: Optional[torch.Tensor], num_adapters: int, tok: int,
+                  slice_offsets: Optional[Sequence[int]] = None, ld_base: int = 0,
+                  stream=None) -> int:
+    """Runs the device-side table checks and returns the LORA_BAD_* bitmask
+    (0 = valid).  Synchronises the stream to read the result."""
+    nseg = seg_indptr.numel() - 1
+    dev = seg_indptr.device
+    result = torch.empty(1, dtype=torch.int32, device=dev)
+    ws = torch.empty(max(int(lib().lora_validate_workspace_size(tok)), 4), dtype=torch.uint8,
+                     device=dev)
+    if slice_offsets is not None:
+        off = [int(v) for v in slice_offsets]
+        S = len(off) - 1
+        off_ptr = ctypes.cast((ctypes.c_int32 * len(off))(*off), ctypes.c_void_p)
+    else:
+        S, off_ptr = 1, None
+    st = lib().lora_validate(_table(seg_indptr, "seg_indptr"), _table(weight_indices,
+                                                                      "weight_indices"),
+                             _table(permutation, "permutation", True), off_ptr, tok, nseg,
+                             num_adapters, S, ld_base, result.data_ptr(), ws.data_ptr(),
+                             ws.numel(), _stream(stream))
+    if st != LORA_OK:
+        raise LoraError("lora_validate", st)
+    (torch.cuda.current_stream() if stream is None else stream).synchronize()
+    return int(result.item())

@@ -1,0 +1,128 @@
+"""The C ABI library loads, exports every declared entry point and rejects bad
+arguments before touching the GPU.  Runs on a machine without a GPU: every
+call here returns before any CUDA call (argument errors, empty problems,
+size queries)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from scatter_gemm_b200 import lora
+from scatter_gemm_b200.build import LIB, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lora_sgmv.h")
+
+OK, INVALID, UNSUPPORTED = 0, 1, 2
+# fake but aligned addresses: the calls below must reject or no-op before use
+P = 0x10000
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return lora.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"LORA_API\s+[\w\s\*]+?\b(lora_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_calls():
+    syms = declared_symbols()
+    for s in ("lora_shrink", "lora_expand", "lora_validate", "lora_status_string",
+              "lora_workspace_size"):
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(L):
+    lib = ctypes.CDLL(LIB)
+    for s in declared_symbols():
+        assert hasattr(lib, s), f"{s} is declared in lora_sgmv.h but not exported"
+
+
+def test_status_strings(L):
+    for code in range(5):
+        assert lora.status_string(code)
+    assert lora.status_string(99) == "unknown status"
+
+
+def shrink(lib, **kw):
+    a = dict(x=P, ld_x=64, A=P, si=P, wi=P, pm=P, out=P, ld_out=48, tok=10, K=64, S=3, r=16,
+             rs=16, nseg=2, nad=4, dt=0, ws=None, wsb=0, st=None)
+    a.update(kw)
+    return lib.lora_shrink(a["x"], a["ld_x"], a["A"], a["si"], a["wi"], a["pm"], a["out"],
+                           a["ld_out"], a["tok"], a["K"], a["S"], a["r"], a["rs"], a["nseg"],
+                           a["nad"], a["dt"], a["ws"], a["wsb"], a["st"])
+
+
+def expand(lib, off=(0, 32, 40, 48), **kw):
+    arr = (ctypes.c_int32 * len(off))(*off)
+    a = dict(inr=P, ld_in=48, B=P, si=P, wi=P, pm=P, offp=ctypes.cast(arr, ctypes.c_void_p),
+             sc=P, base=P, ld_base=48, tok=10, S=len(off) - 1, r=16, rs=16, nseg=2, nad=4, dt=0,
+             ws=None, wsb=0, st=None)
+    a.update(kw)
+    return lib.lora_expand(a["inr"], a["ld_in"], a["B"], a["si"], a["wi"], a["pm"], a["offp"],
+                           a["sc"], a["base"], a["ld_base"], a["tok"], a["S"], a["r"], a["rs"],
+                           a["nseg"], a["nad"], a["dt"], a["ws"], a["wsb"], a["st"])
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(x=None), INVALID), (dict(A=None), INVALID), (dict(si=None), INVALID),
+    (dict(wi=None), INVALID), (dict(out=None), INVALID),
+    (dict(tok=-1), INVALID), (dict(nseg=-1), INVALID), (dict(K=0), INVALID),
+    (dict(S=0), INVALID), (dict(r=0), INVALID), (dict(rs=8), INVALID), (dict(nad=0), INVALID),
+    (dict(S=9, ld_out=9 * 16), UNSUPPORTED), (dict(dt=2), UNSUPPORTED),
+    (dict(ld_x=63), INVALID), (dict(ld_out=47), INVALID),
+    (dict(wsb=16), INVALID),  # workspace bytes without a workspace
+    (dict(x=P + 1), INVALID), (dict(out=P + 1), INVALID), (dict(si=P + 2), INVALID),
+    (dict(pm=P + 2), INVALID),
+    (dict(tok=0), OK), (dict(nseg=0), OK), (dict(tok=0, pm=None), OK),
+])
+def test_shrink_argument_checks(L, kw, want):
+    assert shrink(L, **kw) == want
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(inr=None), INVALID), (dict(B=None), INVALID), (dict(sc=None), INVALID),
+    (dict(base=None), INVALID), (dict(offp=None), INVALID),
+    (dict(r=17), INVALID), (dict(ld_in=47), INVALID), (dict(dt=7), UNSUPPORTED),
+    (dict(ld_base=47), INVALID),  # off[S] > ld_base
+    (dict(sc=P + 2), INVALID), (dict(base=P + 1), INVALID),
+    (dict(tok=0), OK), (dict(nseg=0), OK),
+])
+def test_expand_argument_checks(L, kw, want):
+    assert expand(L, **kw) == want
+
+
+def test_expand_rejects_bad_slice_tables(L):
+    assert expand(L, off=(0, 40, 32, 48)) == INVALID      # decreasing
+    assert expand(L, off=(-1, 32, 40, 48)) == INVALID     # negative
+    assert expand(L, off=(0, 32, 40, 48), ld_base=40) == INVALID
+    assert expand(L, off=tuple(range(0, 80, 8)), ld_in=9 * 16) == UNSUPPORTED  # S = 9
+    assert expand(L, off=(8, 8), S=1, tok=5) == OK        # no columns: nothing to do
+
+
+def test_workspace_sizes(L):
+    assert lora.workspace_size(0, 0, 1) > 0
+    assert lora.workspace_size(8192, 1024, 64) >= 4 * (8192 + 65)
+    assert L.lora_validate_workspace_size(1000) >= 4 * 32
+    assert L.lora_workspace_size(-1, 0, 1) == 0
+
+
+def test_validate_argument_checks(L):
+    res = P
+    assert L.lora_validate(None, P, P, None, 10, 2, 4, 1, 0, res, P, 64, None) == INVALID
+    assert L.lora_validate(P, P, P, None, 10, 2, 4, 1, 0, None, P, 64, None) == INVALID
+    # a permutation needs scratch for its bijection check
+    assert L.lora_validate(P, P, P, None, 10, 2, 4, 1, 0, res, None, 0, None) == INVALID
+    assert L.lora_validate(P, P, P, None, 100, 2, 4, 1, 0, res, P, 4, None) == INVALID
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(lora, "_lib", None)
+    monkeypatch.setattr(lora, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        lora.lib()
