@@ -80,6 +80,14 @@ enum {
   LORA_BAD_SLICES = 16      /* slice_offsets negative, decreasing or > ld_base */
 };
 
+/* Kernel path bits reported by lora_last_path. */
+enum {
+  LORA_PATH_GENERAL = 1, /* element-aligned CUDA-core kernel                       */
+  LORA_PATH_TENSOR = 2,  /* tcgen05 tensor-core kernel (16-byte-aligned inputs)     */
+  LORA_PATH_GROUPED = 4, /* rows grouped by adapter first (workspace, many segments) */
+  LORA_PATH_SPLITK = 8   /* shrink K range split over a thread-block cluster        */
+};
+
 /* Limits of this build. */
 #define LORA_MAX_SLICES 8
 
@@ -154,6 +162,17 @@ LORA_API lora_status lora_validate(const int32_t* seg_indptr, const int32_t* wei
                           void* stream);
 
 LORA_API size_t lora_validate_workspace_size(int tok);
+
+/* Kernel path (LORA_PATH_* bits) chosen by the last lora_shrink / lora_expand
+ * call made on this host thread; 0 if none launched a kernel. */
+LORA_API int lora_last_path(void);
+
+/* Failure detection of the tensor-core kernels.  Every wait inside them is
+ * bounded (1 s); a wait that runs out records a nonzero code in a device word,
+ * and the kernel releases its resources and returns without further writes.
+ * This call reads that word (synchronously, on the current device) into *code
+ * and clears it if `clear` is nonzero. */
+LORA_API lora_status lora_device_error(int32_t* code, int clear);
 
 /* Static description of a status code; never NULL. */
 LORA_API const char* lora_status_string(lora_status status);

@@ -1,0 +1,311 @@
+// expand_tc.cuh -- tensor-core expand with a fused scale-and-add scatter
+// epilogue, for 16-byte-aligned inputs (sm_100a).
+//
+// One CTA handles one piece (<= 128 sorted rows of one segment) times a run of
+// 128-column tiles of the base output.  For every tile (slice q, columns
+// [c0, c0+128) inside the slice):
+//     D[128 x 128] = R_q[128 x r] * B_a[c0-off0 : c0-off0+128, 0:r]^T
+// on tcgen05.mma (M = 128 tokens, N = 128 columns, K = r padded to 16/32/64)
+// with a double-buffered fp32 accumulator in TMEM, and then
+//     base[perm[row], c] = round(base[perm[row], c] + scaling[a] * D[row, c]).
+// This is the expand and the "scatter epilogue" of the sgl-kernel-xpu page
+// ("Decode LoRA kernels are optimized", section "Summary"), rebuilt for B200.
+//
+// Data movement: the rank activations of the piece (all S slices) are loaded
+// once with cp.async, whose partial-size form zero-fills the storage padding
+// j >= r; B tiles come by TMA (the tensor map's inner extent is r, so columns
+// j >= r read as zero); base tiles stream through a ring of shared-memory
+// stages with coalesced 16-byte cp.async (two rows of 256 bytes per warp
+// instruction), are updated in place by the thread that owns the row's
+// accumulator (TMEM lane = row), and are written back with coalesced 16-byte
+// stores.  The 16-byte chunks of a staged base row are XOR-swizzled by the
+// row index, so both the row-per-thread phase and the coalesced phases are
+// free of shared-memory bank conflicts.
+#pragma once
+
+#include "common.cuh"
+#include "general.cuh"
+#include "sched.cuh"
+#include "sm100.cuh"
+
+namespace lora {
+
+constexpr int kExBM = 128;      // rows per piece
+constexpr int kExBN = 128;      // columns per tile
+constexpr int kExThreads = 160;
+constexpr int kExTileBytes = kExBM * kExBN * 2;  // staged base tile
+
+struct ExpandTcParams {
+  CUtensorMap tmap_B;  // 2-D [L*N_tot rows, r cols] (row stride rs), box {rpad, 128}
+  ExpandArgs a;
+  const int32_t* row_list;     // grouped schedule (or null)
+  const int32_t* vseg_indptr;  // grouped schedule (or null)
+  int nvseg;
+  int rpad;                    // 16, 32 or 64
+  int tiles_total;             // 128-column tiles over all slices
+  int tiles_per_cta;
+  int tile_prefix[LORA_MAX_SLICES + 1];  // first tile of each slice
+  int base_stages;             // ring depth of base tiles
+  int b_stages;                // ring depth of B tiles
+  uint32_t idesc;
+  uint32_t sw_layout;          // UMMA layout code of rows of rpad*2 bytes
+  uint32_t rin_bytes;          // one slice of staged rank activations (128 * rpad * 2)
+  uint32_t btile_bytes;        // one B tile (128 * rpad * 2)
+};
+
+// physical 16-byte chunk of logical chunk c in a row of the rank-activation /
+// B tiles (rows of rpad*2 bytes, canonical UMMA swizzle)
+__device__ __forceinline__ int swz_chunk(int c, int m, int rpad) {
+  return rpad == 64 ? (c ^ (m & 7)) : rpad == 32 ? (c ^ ((m >> 1) & 3)) : (c ^ ((m >> 2) & 1));
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+template <class E>
+__global__ void __launch_bounds__(kExThreads, 1)
+expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const ExpandArgs& p = P.a;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int ncg = (P.tiles_total + P.tiles_per_cta - 1) / P.tiles_per_cta;
+  const int slot = blockIdx.x / ncg;
+  const int t_begin = (blockIdx.x % ncg) * P.tiles_per_cta;
+  const int ntl = min(P.tiles_total, t_begin + P.tiles_per_cta) - t_begin;
+
+  Piece pc;
+  const int32_t* indptr = P.vseg_indptr ? P.vseg_indptr : p.seg_indptr;
+  if (ntl <= 0 || !find_piece(indptr, P.nvseg, p.tok, kExBM, slot, pc)) return;
+  const int rows = pc.hi - pc.lo;
+  const int adapter = P.vseg_indptr ? clampi(pc.seg, 0, p.L - 1)
+                                    : clampi(__ldg(p.weight_indices + pc.seg), 0, p.L - 1);
+  const float scale = __ldg(p.scalings + adapter);
+  if (scale == 0.f) return;  // zero scaling: the rows stay bit-identical
+
+  // ---- shared memory: [base ring][rank activations S x][B ring][tok rows][barriers]
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t base_ring = sbase;
+  const uint32_t rin = base_ring + P.base_stages * kExTileBytes;
+  const uint32_t bring = rin + p.S * P.rin_bytes;
+  int* trow = reinterpret_cast<int*>(smem + (bring - sbase) + P.b_stages * P.btile_bytes);
+  int* srow_of = trow + kExBM;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(srow_of + kExBM);
+  const uint32_t bfull0 = smem_u32(bars);
+  const uint32_t bempty0 = bfull0 + 8 * P.b_stages;
+  const uint32_t tfull0 = bempty0 + 8 * P.b_stages;   // 2 accumulator buffers
+  const uint32_t tempty0 = tfull0 + 16;
+  const uint32_t rin_bar = tempty0 + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * P.b_stages + 5);
+
+  const int off0 = p.slices.off[0];
+  const int64_t n_tot = p.slices.off[p.S] - off0;
+
+  if (tid < kExBM) {
+    const int m = tid;
+    int sr = pc.lo + (m < rows ? m : 0);
+    if (P.row_list) sr = clampi(__ldg(P.row_list + sr), 0, p.tok - 1);
+    srow_of[m] = sr;
+    trow[m] = p.permutation ? clampi(__ldg(p.permutation + sr), 0, p.tok - 1) : sr;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < P.b_stages; ++s) {
+      mbar_init(bfull0 + 8 * s, 1);
+      mbar_init(bempty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, kExBM);
+    }
+    mbar_init(rin_bar, kExBM);
+    fence_mbar_init();
+    tma_prefetch_desc(&P.tmap_B);
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+
+  // tile t of this CTA -> (slice, first column)
+  auto tile_info = [&](int t, int& q, int& c0) {
+    const int g = t_begin + t;
+    q = 0;
+#pragma unroll
+    for (int k = 1; k < LORA_MAX_SLICES; ++k)
+      if (k < p.S && g >= P.tile_prefix[k]) q = k;
+    c0 = p.slices.off[q] + (g - P.tile_prefix[q]) * kExBN;
+  };
+
+  if (warp == 4) {
+    // =========================== B tiles (TMA) and MMA issue
+    if (lane == 0) {
+      const int pre = min(P.b_stages, ntl);
+      for (int t = 0; t < pre; ++t) {
+        int q, c0;
+        tile_info(t, q, c0);
+        mbar_arrive_expect_tx(bfull0 + 8 * t, P.btile_bytes);
+        tma_load_2d(bring + t * P.btile_bytes, &P.tmap_B, bfull0 + 8 * t, 0,
+                    static_cast<int>(adapter * n_tot + (c0 - off0)));
+      }
+      ok = mbar_wait(rin_bar, 0);
+      for (int t = 0; t < ntl && ok; ++t) {
+        const int s = t % P.b_stages, buf = t & 1;
+        if (t >= 2) ok = mbar_wait(tempty0 + 8 * buf, ((t - 2) >> 1) & 1);
+        if (ok) ok = mbar_wait(bfull0 + 8 * s, (t / P.b_stages) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        int q, c0;
+        tile_info(t, q, c0);
+        const uint32_t a_s = rin + q * P.rin_bytes;
+        const uint32_t b_s = bring + s * P.btile_bytes;
+        for (int kk = 0; kk < P.rpad / 16; ++kk) {
+          const uint64_t ad = make_sdesc(a_s + kk * 32, P.rpad * 2, P.sw_layout);
+          const uint64_t bd = make_sdesc(b_s + kk * 32, P.rpad * 2, P.sw_layout);
+          tc_mma_f16(tmem + buf * kExBN, ad, bd, P.idesc, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(tfull0 + 8 * buf);
+        tc_commit(bempty0 + 8 * s);
+        // refill the slot of tile t-1 with tile t-1+b_stages
+        const int tn = t - 1 + P.b_stages;
+        if (t >= 1 && tn < ntl) {
+          const int sp = (t - 1) % P.b_stages;
+          ok = mbar_wait(bempty0 + 8 * sp, ((t - 1) / P.b_stages) & 1);
+          if (!ok) break;
+          int q2, c2;
+          tile_info(tn, q2, c2);
+          mbar_arrive_expect_tx(bfull0 + 8 * sp, P.btile_bytes);
+          tma_load_2d(bring + sp * P.btile_bytes, &P.tmap_B, bfull0 + 8 * sp, 0,
+                      static_cast<int>(adapter * n_tot + (c2 - off0)));
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // =========================== rank activations, base stream, epilogue (128 threads)
+    const int m = tid;  // accumulator row of this thread
+    // (1) rank activations of every slice, zero-filled beyond r
+    {
+      const int sr = srow_of[m];
+      const bool row_ok = m < rows;
+      const int nchunk = P.rpad / 8;
+      for (int q = 0; q < p.S; ++q) {
+        const uint16_t* src = p.in_r + static_cast<int64_t>(sr) * p.ld_in + q * p.rs;
+        for (int c = 0; c < nchunk; ++c) {
+          const int left = p.r - 8 * c;
+          const uint32_t nb = row_ok ? static_cast<uint32_t>(max(0, min(left, 8)) * 2) : 0u;
+          const uint32_t dst = rin + q * P.rin_bytes + m * (P.rpad * 2) +
+                               (swz_chunk(c, m, P.rpad) << 4);
+          cp_async_16(dst, nb ? static_cast<const void*>(src + 8 * c)
+                              : static_cast<const void*>(p.in_r), nb);
+        }
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      mbar_arrive(rin_bar);
+    }
+
+    // (2) base tile loads: chunk u = j*128 + tid -> row u/16, logical chunk u%16
+    auto load_base = [&](int t) {
+      int q, c0;
+      tile_info(t, q, c0);
+      const int cend = p.slices.off[q + 1];
+      const uint32_t stage = base_ring + (t % P.base_stages) * kExTileBytes;
+#pragma unroll 4
+      for (int j = 0; j < (kExBM * 16) / kExBM; ++j) {
+        const int u = j * kExBM + m;
+        const int row = u >> 4, c = u & 15;
+        const int col = c0 + 8 * c;
+        const bool in = row < rows && col < cend;
+        const uint16_t* src = p.base + static_cast<int64_t>(trow[row]) * p.ld_base + col;
+        cp_async_16(stage + row * 256 + ((c ^ (row & 15)) << 4),
+                    in ? static_cast<const void*>(src) : static_cast<const void*>(p.base),
+                    in ? 16u : 0u);
+      }
+    };
+    const int pre = min(P.base_stages - 1, ntl);
+    for (int t = 0; t < P.base_stages - 1; ++t) {
+      if (t < pre) load_base(t);
+      cp_async_commit();
+    }
+
+    for (int t = 0; t < ntl; ++t) {
+      const int buf = t & 1;
+      if (t + P.base_stages - 1 < ntl) load_base(t + P.base_stages - 1);
+      cp_async_commit();
+      cp_async_wait_dyn(P.base_stages - 1);  // this thread's copies of tile t have landed
+      named_bar_sync(1, kExBM);              // ... and everybody else's
+      if (ok) ok = mbar_wait(tfull0 + 8 * buf, (t >> 1) & 1);
+      ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+      tc_fence_after();
+      int q, c0;
+      tile_info(t, q, c0);
+      const uint32_t stage = base_ring + (t % P.base_stages) * kExTileBytes;
+      uint8_t* stage_p = smem + (stage - sbase);
+      const uint32_t tacc = tmem + (static_cast<uint32_t>(warp * 32) << 16) + buf * kExBN;
+      // (3) row-per-thread: base + scaling * acc, in place in shared memory
+#pragma unroll 1
+      for (int cc = 0; cc < kExBN / 16; ++cc) {
+        float v[16];
+        if (ok) {
+          tmem_ld16(tacc + cc * 16, v);
+          tmem_ld_wait();
+        }
+        if (ok && m < rows) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int c = 2 * cc + h;
+            uint4* ptr = reinterpret_cast<uint4*>(stage_p + m * 256 + ((c ^ (m & 15)) << 4));
+            uint4 w = *ptr;
+            uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 b = E::u32_to_f2(wv[e]);
+              wv[e] = E::f2_to_u32(fmaf(scale, v[8 * h + 2 * e], b.x),
+                                   fmaf(scale, v[8 * h + 2 * e + 1], b.y));
+            }
+            *ptr = w;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty0 + 8 * buf);
+      named_bar_sync(1, kExBM);
+      // (4) coalesced write-back
+      const int cend = p.slices.off[q + 1];
+      if (ok) {
+#pragma unroll 4
+        for (int j = 0; j < 16; ++j) {
+          const int u = j * kExBM + m;
+          const int row = u >> 4, c = u & 15;
+          const int col = c0 + 8 * c;
+          if (row < rows && col < cend) {
+            const uint4 w = *reinterpret_cast<const uint4*>(stage_p + row * 256 +
+                                                            ((c ^ (row & 15)) << 4));
+            *reinterpret_cast<uint4*>(p.base + static_cast<int64_t>(trow[row]) * p.ld_base +
+                                      col) = w;
+          }
+        }
+      }
+      named_bar_sync(1, kExBM);  // the stage may be refilled
+    }
+    cp_async_wait<0>();
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace lora

@@ -1,0 +1,92 @@
+// group.cuh -- adapter-grouped schedule for tables with many small segments.
+//
+// The sgl-kernel-xpu page ("Decode LoRA kernels are optimized", section
+// "Behaviour changes") asks callers to pass one coalesced segment per adapter
+// because the kernels tile M themselves.  When a caller does not (here: more
+// segments than adapters and a workspace to work in), this single-CTA pass
+// coalesces on the device instead: it lists the rows of every adapter's
+// segments contiguously, so the tensor-core kernels tile each adapter's rows
+// in 128-row pieces and read each adapter's weights once per piece instead of
+// once per segment.  Nothing is synchronised with the host.
+//
+// Workspace layout (int32): vseg_indptr[L+1] | seg_base[nseg] | row_list[tok]
+//   vseg_indptr  rows of adapter a are grouped rows [vseg_indptr[a], vseg_indptr[a+1])
+//   row_list     grouped row g -> sorted row i (and so token permutation[i])
+// The order of segments inside one adapter's group follows an atomic
+// counter; each output row's value does not depend on it.
+#pragma once
+
+#include "common.cuh"
+#include "sched.cuh"
+
+namespace lora {
+
+constexpr int kGroupThreads = 1024;
+constexpr int kGroupMaxAdapters = 8192;
+
+__global__ void __launch_bounds__(kGroupThreads)
+group_rows_kernel(const int32_t* __restrict__ seg_indptr, const int32_t* __restrict__ weight_indices,
+                  int nseg, int L, int tok, int32_t* __restrict__ vseg_indptr,
+                  int32_t* __restrict__ seg_base, int32_t* __restrict__ row_list) {
+  extern __shared__ int cnt[];  // [L] counts, then cursors
+  __shared__ int warp_tot[32];
+  const int tid = threadIdx.x;
+  for (int a = tid; a < L; a += blockDim.x) cnt[a] = 0;
+  __syncthreads();
+  for (int s = tid; s < nseg; s += blockDim.x) {
+    const int lo = clampi(seg_indptr[s], 0, tok), hi = clampi(seg_indptr[s + 1], 0, tok);
+    if (hi > lo) atomicAdd(&cnt[clampi(weight_indices[s], 0, L - 1)], hi - lo);
+  }
+  __syncthreads();
+
+  // exclusive scan of cnt[0..L) -> vseg_indptr and cursors (block-wide, chunked)
+  const int per = (L + blockDim.x - 1) / blockDim.x;
+  const int a0 = tid * per, a1 = min(L, a0 + per);
+  int local = 0;
+  for (int a = a0; a < a1; ++a) local += cnt[a];
+  // inclusive scan of `local` over the block
+  const int lane = tid & 31, wid = tid >> 5;
+  int v = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) warp_tot[wid] = v;
+  __syncthreads();
+  if (wid == 0) {
+    int w = lane < (blockDim.x >> 5) ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += n;
+    }
+    warp_tot[lane] = w;  // inclusive prefix of warp totals
+  }
+  __syncthreads();
+  int run = v - local + (wid > 0 ? warp_tot[wid - 1] : 0);  // exclusive prefix of this thread
+  for (int a = a0; a < a1; ++a) {
+    const int c = cnt[a];
+    vseg_indptr[a] = run;
+    cnt[a] = run;  // becomes the cursor of adapter a
+    run += c;
+  }
+  if (tid == blockDim.x - 1) vseg_indptr[L] = run;
+  __syncthreads();
+
+  for (int s = tid; s < nseg; s += blockDim.x) {
+    const int lo = clampi(seg_indptr[s], 0, tok), hi = clampi(seg_indptr[s + 1], 0, tok);
+    seg_base[s] = hi > lo ? atomicAdd(&cnt[clampi(weight_indices[s], 0, L - 1)], hi - lo) : 0;
+  }
+  __syncthreads();
+
+  const int rlo = clampi(seg_indptr[0], 0, tok), rhi = clampi(seg_indptr[nseg], 0, tok);
+  for (int i = rlo + tid; i < rhi; i += blockDim.x) {
+    const int s = count_le(seg_indptr, nseg + 1, i) - 1;
+    if (s < 0 || s >= nseg) continue;
+    const int g = seg_base[s] + (i - clampi(seg_indptr[s], 0, tok));
+    if (g >= 0 && g < tok) row_list[g] = i;
+  }
+}
+
+}  // namespace lora

@@ -3,19 +3,38 @@
 // "Decode LoRA kernels are optimized", sections "Summary" and "Behaviour
 // changes").  Nothing here reads a device table on the host and nothing is
 // synchronised: every call enqueues its kernels on the caller's stream.
+//
+// Kernel selection (run time, from pointers and sizes only):
+//   tensor-core kernels (shrink_tc / expand_tc) when every tensor they stream
+//   is 16-byte aligned with 16-byte-multiple row strides, K % 8 == 0, the
+//   padded shrink width S*rs <= 256, slice starts % 8 == 0 and r <= 64 for the
+//   expand; otherwise the element-aligned CUDA-core kernels of general.cuh.
+//   With a workspace and more segments than adapters the tensor-core kernels
+//   run on the adapter-grouped schedule of group.cuh.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/lora_sgmv.h"
 #include "common.cuh"
+#include "expand_tc.cuh"
 #include "general.cuh"
+#include "group.cuh"
 #include "sched.cuh"
+#include "shrink_tc.cuh"
+#include "sm100.cuh"
 
 namespace {
 
 thread_local uint64_t g_launches = 0;
+thread_local int g_last_path = 0;
+
+constexpr int kMaxDevices = 64;
 
 inline bool aligned_to(const void* p, uintptr_t a) {
   return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
@@ -25,6 +44,139 @@ inline lora_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
 }
 
+inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
+
+// ------------------------------------------------------------------ device facts
+
+struct DeviceFacts {
+  std::atomic<int> ready{0};
+  int sms = 148;
+  int max_cluster = 8;  // largest K-split cluster the shrink may use
+};
+DeviceFacts g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+template <class E>
+void set_kernel_attrs() {
+  cudaFuncSetAttribute(lora::shrink_tc_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       227 * 1024);
+  cudaFuncSetAttribute(lora::shrink_tc_kernel<E>,
+                       cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaFuncSetAttribute(lora::expand_tc_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       227 * 1024);
+  cudaFuncSetAttribute(lora::expand_general_kernel<E>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+}
+
+const DeviceFacts* device_facts() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  DeviceFacts& f = g_dev[dev];
+  if (f.ready.load(std::memory_order_acquire)) return &f;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!f.ready.load(std::memory_order_relaxed)) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return nullptr;
+    f.sms = sms;
+    set_kernel_attrs<lora::Bf16>();
+    set_kernel_attrs<lora::Fp16>();
+    // can 16 CTAs of the shrink (at its largest two-per-SM footprint) form a cluster?
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 16;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(16 * 16);
+    cfg.blockDim = dim3(lora::kTcThreads);
+    cfg.dynamicSmemBytes = 112 * 1024;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int nclusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, lora::shrink_tc_kernel<lora::Bf16>, &cfg) ==
+            cudaSuccess &&
+        nclusters > 0)
+      f.max_cluster = 16;
+    cudaGetLastError();  // the probe above must not leave a sticky launch error
+    f.ready.store(1, std::memory_order_release);
+  }
+  return &f;
+}
+
+// ------------------------------------------------------------------ TMA tensor maps
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor of 16-bit elements: `cols` valid columns, `rows` rows,
+// `row_bytes` between rows; box {box_cols, box_rows}.
+bool encode_2d(CUtensorMap* m, lora_dtype dt, const void* base, uint64_t cols, uint64_t rows,
+               uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows,
+               CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, dt == LORA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                            : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ workspace
+
+struct Grouping {
+  const int32_t* vseg_indptr = nullptr;
+  const int32_t* row_list = nullptr;
+  int nvseg = 0;
+};
+
+inline size_t a16(size_t n) { return (n + 3) / 4 * 4; }  // ints -> multiple of 4 ints
+
+size_t workspace_ints(int tok, int nseg, int L) {
+  return a16(static_cast<size_t>(L) + 1) + a16(static_cast<size_t>(nseg)) +
+         a16(static_cast<size_t>(tok));
+}
+
+// Enqueues the grouping pass when the schedule calls for it.
+lora_status maybe_group(const int32_t* seg_indptr, const int32_t* weight_indices, int tok,
+                        int nseg, int L, void* ws, size_t ws_bytes, cudaStream_t st,
+                        Grouping& g) {
+  g = Grouping{};
+  if (!ws || nseg <= L || L > lora::kGroupMaxAdapters) return LORA_OK;
+  if (!aligned_to(ws, 16) || ws_bytes < workspace_ints(tok, nseg, L) * 4) return LORA_OK;
+  int32_t* w = static_cast<int32_t*>(ws);
+  int32_t* vseg = w;
+  int32_t* seg_base = vseg + a16(static_cast<size_t>(L) + 1);
+  int32_t* rows = seg_base + a16(static_cast<size_t>(nseg));
+  lora::group_rows_kernel<<<1, lora::kGroupThreads, sizeof(int) * L, st>>>(
+      seg_indptr, weight_indices, nseg, L, tok, vseg, seg_base, rows);
+  ++g_launches;
+  if (launch_status() != LORA_OK) return LORA_ERR_CUDA;
+  g.vseg_indptr = vseg;
+  g.row_list = rows;
+  g.nvseg = L;
+  return LORA_OK;
+}
+
+// ------------------------------------------------------------------ shrink
+
 template <class E>
 lora_status shrink_general(const lora::ShrinkArgs& a, cudaStream_t st) {
   const int slots = lora::num_piece_slots(a.tok, a.nseg, lora::kGBM);
@@ -33,8 +185,75 @@ lora_status shrink_general(const lora::ShrinkArgs& a, cudaStream_t st) {
   dim3 grid(slots, groups);
   lora::shrink_general_kernel<E><<<grid, lora::kGWarps * 32, 0, st>>>(a);
   ++g_launches;
+  g_last_path = LORA_PATH_GENERAL;
   return launch_status();
 }
+
+bool shrink_tc_eligible(const lora::ShrinkArgs& a) {
+  const int npad = round_up(a.S * a.rs, 16);
+  return aligned_to(a.x, 16) && (a.ld_x % 8) == 0 && (a.K % 8) == 0 && aligned_to(a.A, 16) &&
+         npad <= 256 && static_cast<int64_t>(a.L) * a.S * a.rs < (int64_t(1) << 31) &&
+         a.tok < (1 << 30);
+}
+
+template <class E>
+lora_status shrink_tc(const lora::ShrinkArgs& a, lora_dtype dt, const Grouping& g,
+                      const DeviceFacts& dev, cudaStream_t st) {
+  lora::ShrinkTcParams P;
+  std::memset(&P, 0, sizeof(P));
+  P.a = a;
+  P.row_list = g.row_list;
+  P.vseg_indptr = g.vseg_indptr;
+  P.nvseg = g.vseg_indptr ? g.nvseg : a.nseg;
+  P.npad = round_up(a.S * a.rs, 16);
+  P.tmem_cols = P.npad <= 32 ? 32 : P.npad <= 64 ? 64 : P.npad <= 128 ? 128 : 256;
+  P.stage_bytes = lora::kTcBM * 128 + P.npad * 128;
+  const int budget = (P.npad <= 128 ? 110 : 200) * 1024;
+  P.stages = (budget - 2048) / static_cast<int>(P.stage_bytes);
+  P.stages = P.stages < 2 ? 2 : (P.stages > 8 ? 8 : P.stages);
+  const size_t part_bytes = sizeof(float) * lora::kTcBM * (P.npad + 1);
+  while (static_cast<size_t>(P.stages) * P.stage_bytes < part_bytes) ++P.stages;
+  P.nkb = (a.K + lora::kTcBK - 1) / lora::kTcBK;
+
+  // K split over a cluster: grow while the grid stays within the resident CTAs
+  const int per_sm = P.npad <= 128 ? 2 : 1;
+  const int target = dev.sms * per_sm;
+  const int est = (a.tok + lora::kTcBM - 1) / lora::kTcBM + (P.vseg_indptr ? a.L : a.nseg) / 2;
+  int cs = 1;
+  while (cs < dev.max_cluster && est * cs * 2 <= target && P.nkb >= 4 * cs) cs *= 2;
+  P.csplit = cs;
+  P.kb_per = (P.nkb + cs - 1) / cs;
+  P.idesc = lora::make_idesc_f16(dt == LORA_BF16 ? 1 : 0, lora::kTcBM, P.npad);
+  if (!encode_2d(&P.tmap_A, dt, a.A, a.K, static_cast<uint64_t>(a.L) * a.S * a.rs,
+                 static_cast<uint64_t>(a.K) * 2, lora::kTcBK, P.npad,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return LORA_ERR_CUDA;
+
+  const size_t smem = static_cast<size_t>(P.stages) * P.stage_bytes + 1024 +
+                      8 * (2 * P.stages + 1) + 16;
+  const long slots = lora::num_piece_slots(a.tok, P.nvseg, lora::kTcBM);
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(static_cast<unsigned>(slots * cs));
+  cfg.blockDim = dim3(lora::kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  if (cs > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, lora::shrink_tc_kernel<E>, P);
+  ++g_launches;
+  g_last_path = LORA_PATH_TENSOR | (cs > 1 ? LORA_PATH_SPLITK : 0) |
+                (P.vseg_indptr ? LORA_PATH_GROUPED : 0);
+  return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ expand
 
 template <class E>
 lora_status expand_general(const lora::ExpandArgs& a, cudaStream_t st) {
@@ -44,16 +263,88 @@ lora_status expand_general(const lora::ExpandArgs& a, cudaStream_t st) {
   if (chunks > 65535) return LORA_ERR_UNSUPPORTED;
   const size_t smem = sizeof(float) * lora::kGBM * a.S * a.r;
   if (smem > 200 * 1024) return LORA_ERR_UNSUPPORTED;
-  if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(lora::expand_general_kernel<E>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return LORA_ERR_CUDA;
-  }
   dim3 grid(slots, chunks);
   lora::expand_general_kernel<E><<<grid, lora::kGECols, smem, st>>>(a);
   ++g_launches;
+  g_last_path = LORA_PATH_GENERAL;
   return launch_status();
+}
+
+bool expand_tc_eligible(const lora::ExpandArgs& a) {
+  if (!(aligned_to(a.in_r, 16) && (a.ld_in % 8) == 0 && (a.rs % 8) == 0 &&
+        aligned_to(a.B, 16) && aligned_to(a.base, 16) && (a.ld_base % 8) == 0 && a.r <= 64))
+    return false;
+  for (int q = 0; q <= a.S; ++q)
+    if (a.slices.off[q] % 8) return false;
+  const int64_t n_tot = a.slices.off[a.S] - a.slices.off[0];
+  return static_cast<int64_t>(a.L) * n_tot < (int64_t(1) << 31) && a.tok < (1 << 30);
+}
+
+template <class E>
+lora_status expand_tc(const lora::ExpandArgs& a, lora_dtype dt, const Grouping& g,
+                      const DeviceFacts& dev, cudaStream_t st) {
+  lora::ExpandTcParams P;
+  std::memset(&P, 0, sizeof(P));
+  P.a = a;
+  P.row_list = g.row_list;
+  P.vseg_indptr = g.vseg_indptr;
+  P.nvseg = g.vseg_indptr ? g.nvseg : a.nseg;
+  P.rpad = a.r <= 16 ? 16 : (a.r <= 32 ? 32 : 64);
+  P.sw_layout = P.rpad == 16 ? 6u : (P.rpad == 32 ? 4u : 2u);
+  const CUtensorMapSwizzle swz = P.rpad == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                 : P.rpad == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                : CU_TENSOR_MAP_SWIZZLE_128B;
+  P.rin_bytes = lora::kExBM * P.rpad * 2;
+  P.btile_bytes = lora::kExBN * P.rpad * 2;
+  int tiles = 0;
+  for (int q = 0; q < a.S; ++q) {
+    P.tile_prefix[q] = tiles;
+    tiles += (a.slices.off[q + 1] - a.slices.off[q] + lora::kExBN - 1) / lora::kExBN;
+  }
+  P.tile_prefix[a.S] = tiles;
+  for (int q = a.S + 1; q <= LORA_MAX_SLICES; ++q) P.tile_prefix[q] = tiles;
+  if (tiles == 0) return LORA_OK;
+  P.tiles_total = tiles;
+  P.idesc = lora::make_idesc_f16(dt == LORA_BF16 ? 1 : 0, lora::kExBM, lora::kExBN);
+
+  // shared memory: base ring, rank activations, B ring, row tables, barriers
+  P.b_stages = 3;
+  const size_t fixed = static_cast<size_t>(a.S) * P.rin_bytes + 1024 + 1024 + 256;
+  P.base_stages = 3;
+  auto total = [&]() {
+    return static_cast<size_t>(P.base_stages) * lora::kExTileBytes + fixed +
+           static_cast<size_t>(P.b_stages) * P.btile_bytes;
+  };
+  if (total() > 113 * 1024) P.base_stages = 2;
+  if (total() > 113 * 1024) P.b_stages = 2;
+  if (total() > 225 * 1024) return LORA_ERR_UNSUPPORTED;
+  size_t smem = total();
+  if (smem < 80 * 1024) smem = 80 * 1024;  // at most two CTAs (2 x 256 TMEM columns) per SM
+
+  const int64_t n_tot = a.slices.off[a.S] - a.slices.off[0];
+  if (!encode_2d(&P.tmap_B, dt, a.B, a.r, static_cast<uint64_t>(a.L) * n_tot,
+                 static_cast<uint64_t>(a.rs) * 2, P.rpad, lora::kExBN, swz))
+    return LORA_ERR_CUDA;
+
+  const long slots = lora::num_piece_slots(a.tok, P.nvseg, lora::kExBM);
+  const long est = (a.tok + lora::kExBM - 1) / lora::kExBM + (P.vseg_indptr ? a.L : a.nseg) / 2;
+  const long target = 2L * dev.sms;
+  long tpc = (est * tiles + target - 1) / target;
+  if (tpc < 1) tpc = 1;
+  if (tpc > tiles) tpc = tiles;
+  P.tiles_per_cta = static_cast<int>(tpc);
+  const long ncg = (tiles + tpc - 1) / tpc;
+  if (slots * ncg >= (1L << 31)) return LORA_ERR_UNSUPPORTED;
+
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(slots * ncg));
+  cfg.blockDim = dim3(lora::kExThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, lora::expand_tc_kernel<E>, P);
+  ++g_launches;
+  g_last_path = LORA_PATH_TENSOR | (P.vseg_indptr ? LORA_PATH_GROUPED : 0);
+  return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
 }
 
 }  // namespace
@@ -73,16 +364,30 @@ const char* lora_status_string(lora_status s) {
 
 uint64_t lora_launch_count(void) { return g_launches; }
 void lora_reset_launch_count(void) { g_launches = 0; }
+int lora_last_path(void) { return g_last_path; }
 
 size_t lora_workspace_size(int tok, int nseg, int L) {
   if (tok < 0 || nseg < 0 || L < 1) return 0;
-  // adapter-grouped schedule: grouped row list + per-adapter row offsets
-  return sizeof(int32_t) * (static_cast<size_t>(tok) + static_cast<size_t>(L) + 1 + 64);
+  return workspace_ints(tok, nseg, L) * sizeof(int32_t);
 }
 
 size_t lora_validate_workspace_size(int tok) {
   if (tok < 0) return 0;
   return sizeof(uint32_t) * ((static_cast<size_t>(tok) + 31) / 32 + 1);
+}
+
+lora_status lora_device_error(int32_t* code, int clear) {
+  if (!code) return LORA_ERR_INVALID_ARGUMENT;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, lora::g_lora_device_error, sizeof(int)) != cudaSuccess)
+    return LORA_ERR_CUDA;
+  *code = v;
+  if (clear) {
+    const int z = 0;
+    if (cudaMemcpyToSymbol(lora::g_lora_device_error, &z, sizeof(int)) != cudaSuccess)
+      return LORA_ERR_CUDA;
+  }
+  return LORA_OK;
 }
 
 lora_status lora_shrink(const void* x, int64_t ld_x, const void* A_stack,
@@ -94,21 +399,31 @@ lora_status lora_shrink(const void* x, int64_t ld_x, const void* A_stack,
   if (tok < 0 || nseg < 0 || K < 1 || S < 1 || r < 1 || rs < r || L < 1)
     return LORA_ERR_INVALID_ARGUMENT;
   if (S > LORA_MAX_SLICES) return LORA_ERR_UNSUPPORTED;
-  if (!x || !A_stack || !seg_indptr || !weight_indices || !out_r)
-    return LORA_ERR_INVALID_ARGUMENT;
   if (ld_x < K || ld_out < static_cast<int64_t>(S) * rs) return LORA_ERR_INVALID_ARGUMENT;
   if (workspace_bytes > 0 && !workspace) return LORA_ERR_INVALID_ARGUMENT;
+  if (tok == 0 || nseg == 0) return LORA_OK;  // nothing to read or write
+  if (!x || !A_stack || !seg_indptr || !weight_indices || !out_r)
+    return LORA_ERR_INVALID_ARGUMENT;
   if (!aligned_to(x, 2) || !aligned_to(A_stack, 2) || !aligned_to(out_r, 2) ||
       !aligned_to(seg_indptr, 4) || !aligned_to(weight_indices, 4) ||
       (permutation && !aligned_to(permutation, 4)))
     return LORA_ERR_INVALID_ARGUMENT;
-  if (tok == 0 || nseg == 0) return LORA_OK;
 
   lora::ShrinkArgs a{static_cast<const uint16_t*>(x), ld_x,
                      static_cast<const uint16_t*>(A_stack), seg_indptr, weight_indices,
                      permutation, static_cast<uint16_t*>(out_r), ld_out, tok, K, S, r, rs,
                      nseg, L};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const DeviceFacts* dev = device_facts();
+  if (!dev) return LORA_ERR_CUDA;
+  if (shrink_tc_eligible(a)) {
+    Grouping g;
+    const lora_status gs =
+        maybe_group(seg_indptr, weight_indices, tok, nseg, L, workspace, workspace_bytes, st, g);
+    if (gs != LORA_OK) return gs;
+    return dtype == LORA_BF16 ? shrink_tc<lora::Bf16>(a, dtype, g, *dev, st)
+                              : shrink_tc<lora::Fp16>(a, dtype, g, *dev, st);
+  }
   return dtype == LORA_BF16 ? shrink_general<lora::Bf16>(a, st)
                             : shrink_general<lora::Fp16>(a, st);
 }
@@ -123,9 +438,7 @@ lora_status lora_expand(const void* in_r, int64_t ld_in, const void* B_stack,
   if (tok < 0 || nseg < 0 || S < 1 || r < 1 || rs < r || L < 1)
     return LORA_ERR_INVALID_ARGUMENT;
   if (S > LORA_MAX_SLICES) return LORA_ERR_UNSUPPORTED;
-  if (!in_r || !B_stack || !seg_indptr || !weight_indices || !slice_offsets || !scalings ||
-      !base_out)
-    return LORA_ERR_INVALID_ARGUMENT;
+  if (!slice_offsets) return LORA_ERR_INVALID_ARGUMENT;
   if (ld_in < static_cast<int64_t>(S) * rs) return LORA_ERR_INVALID_ARGUMENT;
   if (workspace_bytes > 0 && !workspace) return LORA_ERR_INVALID_ARGUMENT;
   lora::SliceTable tab{};
@@ -135,17 +448,29 @@ lora_status lora_expand(const void* in_r, int64_t ld_in, const void* B_stack,
     if (slice_offsets[q] < 0 || slice_offsets[q] > ld_base) return LORA_ERR_INVALID_ARGUMENT;
     if (q > 0 && slice_offsets[q] < slice_offsets[q - 1]) return LORA_ERR_INVALID_ARGUMENT;
   }
+  if (tok == 0 || nseg == 0 || tab.off[S] == tab.off[0]) return LORA_OK;
+  if (!in_r || !B_stack || !seg_indptr || !weight_indices || !scalings || !base_out)
+    return LORA_ERR_INVALID_ARGUMENT;
   if (!aligned_to(in_r, 2) || !aligned_to(B_stack, 2) || !aligned_to(base_out, 2) ||
       !aligned_to(seg_indptr, 4) || !aligned_to(weight_indices, 4) ||
       !aligned_to(scalings, 4) || (permutation && !aligned_to(permutation, 4)))
     return LORA_ERR_INVALID_ARGUMENT;
-  if (tok == 0 || nseg == 0 || tab.off[S] == tab.off[0]) return LORA_OK;
 
   lora::ExpandArgs a{static_cast<const uint16_t*>(in_r), ld_in,
                      static_cast<const uint16_t*>(B_stack), seg_indptr, weight_indices,
                      permutation, scalings, static_cast<uint16_t*>(base_out), ld_base, tok, S,
                      r, rs, nseg, L, tab};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const DeviceFacts* dev = device_facts();
+  if (!dev) return LORA_ERR_CUDA;
+  if (expand_tc_eligible(a)) {
+    Grouping g;
+    const lora_status gs =
+        maybe_group(seg_indptr, weight_indices, tok, nseg, L, workspace, workspace_bytes, st, g);
+    if (gs != LORA_OK) return gs;
+    return dtype == LORA_BF16 ? expand_tc<lora::Bf16>(a, dtype, g, *dev, st)
+                              : expand_tc<lora::Fp16>(a, dtype, g, *dev, st);
+  }
   return dtype == LORA_BF16 ? expand_general<lora::Bf16>(a, st)
                             : expand_general<lora::Fp16>(a, st);
 }

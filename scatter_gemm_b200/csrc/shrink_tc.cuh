@@ -1,0 +1,238 @@
+// shrink_tc.cuh -- tensor-core shrink for 16-byte-aligned inputs (sm_100a).
+//
+// One CTA computes one piece (<= 128 sorted rows of one segment, from the
+// scheduler of sched.cuh) times one K range:
+//     D[128 x NPAD] = X_piece[128 x K_range] * A_a[NPAD x K_range]^T
+// with NPAD = S*rs rounded up to 16.  The contraction runs on tcgen05.mma
+// (M = 128, N = NPAD, K = 16 per instruction) with the fp32 accumulator in
+// TMEM.  This is the "gathered-A mainloop" of the sgl-kernel-xpu page
+// ("Decode LoRA kernels are optimized", section "Summary"), rebuilt for B200:
+//
+//  - warps 0-3 gather the piece's x rows (row m = token perm[lo+m]) with
+//    16-byte cp.async straight into the 128-byte-swizzled K-major layout the
+//    MMA reads, K block by K block (64 elements), through a ring of stages;
+//  - thread 0 loads the adapter's A block of the stage with one TMA tiled
+//    copy (rows a*S*rs ... + NPAD, 64 K columns; out-of-range rows and K
+//    columns are zero-filled by the TMA unit);
+//  - warp 4 issues the MMAs and returns each stage with tcgen05.commit;
+//  - warps 0-3 then read the accumulator back (tcgen05.ld, one row per
+//    thread) and round each valid column (j < r of every slice) once.
+//
+// Split-K: for small token counts the K range is split over the CTAs of a
+// thread-block cluster (grid = pieces x C, cluster = C CTAs along K).  Each
+// CTA leaves its fp32 partial in its own shared memory; after a cluster
+// barrier CTA c sums rows [c*128/C, (c+1)*128/C) over all C partials through
+// distributed shared memory, in rank order (deterministic), and writes them.
+// No global scratch and no atomics.
+#pragma once
+
+#include "common.cuh"
+#include "general.cuh"
+#include "sched.cuh"
+#include "sm100.cuh"
+
+namespace lora {
+
+constexpr int kTcBM = 128;   // rows per piece (MMA M)
+constexpr int kTcBK = 64;    // K elements per stage (one 128-byte swizzle row)
+constexpr int kTcThreads = 160;
+
+struct ShrinkTcParams {
+  CUtensorMap tmap_A;  // 2-D [L*S*rs rows, K cols], box {64, NPAD}, 128B swizzle
+  ShrinkArgs a;
+  const int32_t* row_list;     // grouped schedule: sorted row of each grouped row (or null)
+  const int32_t* vseg_indptr;  // grouped schedule: rows of each adapter group (or null)
+  int nvseg;                   // number of (virtual) segments the scheduler walks
+  int npad;                    // MMA N
+  int tmem_cols;               // power of two >= npad, >= 32
+  int stages;
+  int nkb;                     // K blocks in total
+  int kb_per;                  // K blocks per split
+  int csplit;                  // CTAs per cluster (K splits)
+  uint32_t idesc;
+  uint32_t stage_bytes;
+};
+
+template <class E>
+__global__ void __launch_bounds__(kTcThreads, 1)
+shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const ShrinkArgs& p = P.a;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int split = blockIdx.x % P.csplit;
+  const int slot = blockIdx.x / P.csplit;
+
+  // ---- piece of this cluster (identical in all its CTAs)
+  Piece pc;
+  const int32_t* indptr = P.vseg_indptr ? P.vseg_indptr : p.seg_indptr;
+  if (!find_piece(indptr, P.nvseg, p.tok, kTcBM, slot, pc)) return;
+  const int rows = pc.hi - pc.lo;
+  const int adapter = P.vseg_indptr ? clampi(pc.seg, 0, p.L - 1)
+                                    : clampi(__ldg(p.weight_indices + pc.seg), 0, p.L - 1);
+
+  // ---- shared memory carve-up (1024-aligned stages, then barriers)
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t x_bytes = kTcBM * 128;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.stages * P.stage_bytes);
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = full0 + 8 * P.stages;
+  const uint32_t done_bar = empty0 + 8 * P.stages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * P.stages + 1);
+
+  const int kb0 = split * P.kb_per;
+  const int nk = max(0, min(P.nkb, kb0 + P.kb_per) - kb0);
+
+  if (tid == 0) {
+    for (int s = 0; s < P.stages; ++s) {
+      mbar_init(full0 + 8 * s, kTcBM + 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(done_bar, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&P.tmap_A);
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(tmem_slot), P.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+
+  if (warp < 4) {
+    // =========================== producer: gather x rows, TMA the A block
+    const int m = tid;  // row of the piece handled by this thread
+    const bool row_ok = m < rows;
+    int srow = pc.lo + (row_ok ? m : 0);
+    if (P.row_list) srow = clampi(__ldg(P.row_list + srow), 0, p.tok - 1);
+    const int t = p.permutation ? clampi(__ldg(p.permutation + srow), 0, p.tok - 1) : srow;
+    const uint16_t* xrow = p.x + static_cast<int64_t>(t) * p.ld_x;
+    const uint32_t a_bytes = P.npad * 128;
+    const int lag = P.stages - 1;
+    for (int i = 0; i < nk && ok; ++i) {
+      const int s = i % P.stages;
+      if (i >= P.stages) ok = mbar_wait(empty0 + 8 * s, ((i / P.stages) - 1) & 1);
+      if (!ok) break;
+      const uint32_t xs = sbase + s * P.stage_bytes;
+      const int k0 = (kb0 + i) * kTcBK;
+      if (tid == 0) {
+        mbar_arrive_expect_tx(full0 + 8 * s, a_bytes);
+        tma_load_2d(xs + x_bytes, &P.tmap_A, full0 + 8 * s, k0, adapter * p.S * p.rs);
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int k = k0 + 8 * c;
+        const bool in = row_ok && k < p.K;
+        const uint32_t dst = xs + m * 128 + ((c ^ (m & 7)) << 4);
+        cp_async_16(dst, in ? static_cast<const void*>(xrow + k) : static_cast<const void*>(p.x),
+                    in ? 16u : 0u);
+      }
+      cp_async_commit();
+      if (i >= lag) {
+        // stage i - lag has landed for this thread: publish it to the MMA (async proxy)
+        cp_async_wait_dyn(lag);
+        fence_proxy_async_smem();
+        mbar_arrive(full0 + 8 * ((i - lag) % P.stages));
+      }
+    }
+    // drain: publish the stages still in flight
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    if (ok) {
+      for (int i = max(0, nk - lag); i < nk; ++i) mbar_arrive(full0 + 8 * (i % P.stages));
+    }
+  } else if (warp == 4) {
+    // =========================== MMA issuer
+    if (lane == 0) {
+      for (int i = 0; i < nk && ok; ++i) {
+        const int s = i % P.stages;
+        ok = mbar_wait(full0 + 8 * s, (i / P.stages) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t xs = sbase + s * P.stage_bytes;
+        const uint32_t as = xs + x_bytes;
+#pragma unroll
+        for (int kk = 0; kk < kTcBK / 16; ++kk) {
+          const uint64_t ad = make_sdesc(xs + kk * 32, 128, 2);
+          const uint64_t bd = make_sdesc(as + kk * 32, 128, 2);
+          tc_mma_f16(tmem, ad, bd, P.idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(empty0 + 8 * s);
+      }
+      if (nk > 0) tc_commit(done_bar); else mbar_arrive(done_bar);
+    }
+    __syncwarp();
+  }
+
+  // =========================== epilogue (warps 0-3: one accumulator row per thread)
+  float* part = reinterpret_cast<float*>(smem);  // split-K partial, reuses the stage ring
+  const int pstride = P.npad + 1;
+  if (warp < 4) {
+    if (ok) ok = mbar_wait(done_bar, 0);
+    ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+    tc_fence_after();
+    const int m = tid;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int nvalid = p.S * p.rs;
+    for (int c0 = 0; c0 < P.npad; c0 += 16) {
+      float v[16];
+      if (nk > 0 && ok) {
+        tmem_ld16(trow + c0, v);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = 0.f;
+      }
+      if (P.csplit == 1) {
+        if (m < rows && ok) {
+          const int orow_i = P.row_list ? clampi(__ldg(P.row_list + pc.lo + m), 0, p.tok - 1)
+                                        : pc.lo + m;
+          uint16_t* orow = p.out + static_cast<int64_t>(orow_i) * p.ld_out;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int n = c0 + i;
+            if (n < nvalid && (n % p.rs) < p.r) orow[n] = E::f32_to_bits(v[i]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) part[m * pstride + c0 + i] = v[i];
+      }
+    }
+    tc_fence_before();
+  }
+
+  if (P.csplit > 1) {
+    cluster_sync();  // every partial of the cluster is in shared memory
+    const int R = kTcBM / P.csplit;
+    const int r0 = split * R;
+    const int nv = p.S * p.r;
+    const uint32_t pbase = smem_u32(part);
+    for (int e = tid; e < R * nv; e += kTcThreads) {
+      const int row = r0 + e / nv;
+      const int v = e % nv;
+      const int n = (v / p.r) * p.rs + (v % p.r);
+      if (row >= rows) continue;
+      const uint32_t off = pbase + 4u * static_cast<uint32_t>(row * pstride + n);
+      float sum = 0.f;
+      for (int q = 0; q < P.csplit; ++q) sum += ld_dsmem_f32(mapa_shared(off, q));
+      const int orow_i = P.row_list ? clampi(__ldg(P.row_list + pc.lo + row), 0, p.tok - 1)
+                                    : pc.lo + row;
+      if (ok) p.out[static_cast<int64_t>(orow_i) * p.ld_out + n] = E::f32_to_bits(sum);
+    }
+    cluster_sync();  // peers are done reading this CTA's partial
+  }
+
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, P.tmem_cols);
+  }
+}
+
+}  // namespace lora

@@ -60,6 +60,10 @@ def lib() -> ctypes.CDLL:
             l.lora_launch_count.restype = ctypes.c_uint64
             l.lora_reset_launch_count.argtypes = []
             l.lora_reset_launch_count.restype = None
+            l.lora_last_path.argtypes = []
+            l.lora_last_path.restype = _I
+            l.lora_device_error.argtypes = [_P, _I]
+            l.lora_device_error.restype = _I
             _lib = l
     return _lib
 
@@ -74,6 +78,23 @@ def launch_count() -> int:
 
 def reset_launch_count() -> None:
     lib().lora_reset_launch_count()
+
+
+PATH_GENERAL, PATH_TENSOR, PATH_GROUPED, PATH_SPLITK = 1, 2, 4, 8
+
+
+def last_path() -> int:
+    """LORA_PATH_* bits of the last call's kernel path on this thread."""
+    return int(lib().lora_last_path())
+
+
+def device_error(clear: bool = True) -> int:
+    """Reads (and clears) the device-side failure code of the bounded waits."""
+    v = ctypes.c_int32(0)
+    st = lib().lora_device_error(ctypes.byref(v), int(clear))
+    if st != LORA_OK:
+        raise LoraError("lora_device_error", st)
+    return int(v.value)
 
 
 def workspace_size(tok: int, nseg: int, num_adapters: int) -> int:

@@ -1,0 +1,102 @@
+"""Tensor-core path coverage: which kernel runs, and parity of the tcgen05
+kernels across their shape classes (MMA N = padded S*rs of 16..256, rank
+paddings 16/32/64 in the expand, split-K cluster sizes 1..16, grouped and
+direct schedules, bf16 and fp16).  Same bar as test_parity_gpu.py."""
+import numpy as np
+import pytest
+
+from scatter_gemm_b200 import lora
+from scatter_gemm_b200.workloads import make_problem
+from tests.test_parity_gpu import check_expand, check_shrink
+
+pytestmark = pytest.mark.gpu
+
+T, G, GEN, SPLIT = lora.PATH_TENSOR, lora.PATH_GROUPED, lora.PATH_GENERAL, lora.PATH_SPLITK
+
+
+def test_aligned_inputs_take_the_tensor_core_path():
+    p = make_problem("qkv", seed=20, tok=256, K=512)
+    check_shrink(p)
+    assert lora.last_path() & T
+    check_expand(p)
+    assert lora.last_path() & T
+
+
+def test_misaligned_inputs_take_the_general_path():
+    p = make_problem("tail", seed=21, tok=100)
+    check_shrink(p)
+    assert lora.last_path() == GEN
+    check_expand(p)
+    assert lora.last_path() == GEN
+
+
+def test_many_segments_with_workspace_are_grouped():
+    p = make_problem("many_small", seed=22, tok=900, nseg=120, K=512, slices=[512, 128, 128])
+    check_shrink(p, workspace=True)
+    assert lora.last_path() & G and lora.last_path() & T
+    check_expand(p, workspace=True)
+    assert lora.last_path() & G and lora.last_path() & T
+    check_shrink(p, workspace=False)
+    assert not lora.last_path() & G
+
+
+def test_small_token_counts_split_k_over_a_cluster():
+    p = make_problem("qkv", seed=23, tok=50, K=4096)
+    check_shrink(p)
+    assert lora.last_path() & SPLIT
+
+
+# shrink shape classes: (S, r, rs) -> MMA N = round_up(S*rs, 16)
+@pytest.mark.parametrize("S,r,rs", [(1, 8, 8), (1, 5, 8), (5, 8, 8), (3, 16, 16), (2, 64, 64),
+                                    (3, 32, 32), (1, 136, 136), (4, 64, 64), (2, 100, 104)])
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_shrink_mma_widths(S, r, rs, dtype):
+    slices = [64 + 8 * q for q in range(S)]
+    p = make_problem("qkv", seed=24 + S + r, tok=333, K=776, slices=slices, r=r, rs=rs,
+                     nseg=6, L=6, recipe="dirichlet", dtype=dtype)
+    check_shrink(p)
+    assert lora.last_path() & T
+
+
+@pytest.mark.parametrize("tok,K", [(7, 64), (40, 4096), (300, 128), (1000, 8), (129, 2056),
+                                   (2048, 6144)])
+def test_shrink_split_k_and_k_tails(tok, K):
+    p = make_problem("qkv", seed=25, tok=tok, K=K, slices=[64, 32, 32])
+    check_shrink(p)
+    assert lora.last_path() & T
+
+
+# expand rank classes: rpad 16 (r<=16), 32 (r<=32), 64 (r<=64)
+@pytest.mark.parametrize("r,rs", [(1, 8), (5, 8), (13, 16), (16, 16), (20, 24), (32, 32),
+                                  (40, 40), (64, 64)])
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_expand_rank_classes(r, rs, dtype):
+    p = make_problem("qkv", seed=26 + r, tok=333, K=64, slices=[1000, 136, 264], r=r, rs=rs,
+                     nseg=5, L=7, recipe="dirichlet", dtype=dtype, col_lead=8, ld_pad=8)
+    check_expand(p)
+    assert lora.last_path() & T
+
+
+@pytest.mark.parametrize("tok", [1, 64, 129, 777, 4100])
+def test_expand_tile_runs_per_cta(tok):
+    p = make_problem("gate_up", seed=27, tok=tok, K=64, slices=[2048, 1288], nseg=4, L=4)
+    check_expand(p)
+    assert lora.last_path() & T
+
+
+def test_expand_empty_slice_and_single_column_tiles():
+    p = make_problem("qkv", seed=28, tok=200, K=64, slices=[128, 0, 8, 120, 0, 136])
+    check_expand(p)
+    assert lora.last_path() & T
+
+
+def test_one_token_per_segment_grouped_and_direct():
+    p = make_problem("ones16k", seed=29, tok=3000, nseg=3000, K=512)
+    check_shrink(p, workspace=True)
+    check_expand(p, workspace=True)
+    check_shrink(p, workspace=False)
+    check_expand(p, workspace=False)
+
+
+def test_no_device_side_wait_timed_out():
+    assert lora.device_error(clear=True) == 0
