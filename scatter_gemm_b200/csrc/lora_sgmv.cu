@@ -29,6 +29,17 @@
 #include "shrink_tc.cuh"
 #include "sm100.cuh"
 
+// Tuning constants of the expand (compile-time; defaults below).
+#ifndef LORA_EXPAND_CTAS_PER_SM
+#define LORA_EXPAND_CTAS_PER_SM 2   // 2: <= 113 KB shared memory per CTA; 1: deeper ring
+#endif
+#ifndef LORA_EXPAND_WAVES
+#define LORA_EXPAND_WAVES 1         // resident-CTA waves the grid is sized for
+#endif
+#ifndef LORA_EXPAND_B_STAGES
+#define LORA_EXPAND_B_STAGES 3
+#endif
+
 namespace {
 
 thread_local uint64_t g_launches = 0;
@@ -215,12 +226,11 @@ lora_status shrink_tc(const lora::ShrinkArgs& a, lora_dtype dt, const Grouping& 
   while (static_cast<size_t>(P.stages) * P.stage_bytes < part_bytes) ++P.stages;
   P.nkb = (a.K + lora::kTcBK - 1) / lora::kTcBK;
 
-  // K split over a cluster: grow while the grid stays within the resident CTAs
-  const int per_sm = P.npad <= 128 ? 2 : 1;
-  const int target = dev.sms * per_sm;
+  // K split over a cluster: the smallest power of two that gives every SM a CTA
+  // (expected pieces: one per 128 rows plus about half a piece per segment)
   const int est = (a.tok + lora::kTcBM - 1) / lora::kTcBM + (P.vseg_indptr ? a.L : a.nseg) / 2;
   int cs = 1;
-  while (cs < dev.max_cluster && est * cs * 2 <= target && P.nkb >= 4 * cs) cs *= 2;
+  while (cs < dev.max_cluster && est * cs < dev.sms && P.nkb >= 8 * cs) cs *= 2;
   P.csplit = cs;
   P.kb_per = (P.nkb + cs - 1) / cs;
   P.idesc = lora::make_idesc_f16(dt == LORA_BF16 ? 1 : 0, lora::kTcBM, P.npad);
@@ -230,7 +240,7 @@ lora_status shrink_tc(const lora::ShrinkArgs& a, lora_dtype dt, const Grouping& 
     return LORA_ERR_CUDA;
 
   const size_t smem = static_cast<size_t>(P.stages) * P.stage_bytes + 1024 +
-                      8 * (2 * P.stages + 1) + 16;
+                      8 * (2 * P.stages + 2) + 8 * lora::kTcBM + 16;
   const long slots = lora::num_piece_slots(a.tok, P.nvseg, lora::kTcBM);
   cudaLaunchConfig_t cfg{};
   cudaLaunchAttribute attr[1];
@@ -308,17 +318,18 @@ lora_status expand_tc(const lora::ExpandArgs& a, lora_dtype dt, const Grouping& 
   P.idesc = lora::make_idesc_f16(dt == LORA_BF16 ? 1 : 0, lora::kExBM, lora::kExBN);
 
   // shared memory: base ring, rank activations, B ring, row tables, barriers
-  P.b_stages = 3;
-  const size_t fixed = static_cast<size_t>(a.S) * P.rin_bytes + 1024 + 1024 + 256;
-  P.base_stages = 3;
-  auto total = [&]() {
-    return static_cast<size_t>(P.base_stages) * lora::kExTileBytes + fixed +
-           static_cast<size_t>(P.b_stages) * P.btile_bytes;
+  P.b_stages = LORA_EXPAND_B_STAGES;
+  const size_t fixed = static_cast<size_t>(a.S) * P.rin_bytes +
+                       static_cast<size_t>(P.b_stages) * P.btile_bytes + 1024 + 1024 + 16;
+  auto total = [&](int bs) {
+    return ((static_cast<size_t>(bs) * lora::kExStageBytes + 1023) & ~size_t(1023)) + fixed +
+           8 * (2 * P.b_stages + 5 + 2 * bs);
   };
-  if (total() > 113 * 1024) P.base_stages = 2;
-  if (total() > 113 * 1024) P.b_stages = 2;
-  if (total() > 225 * 1024) return LORA_ERR_UNSUPPORTED;
-  size_t smem = total();
+  const size_t cap = (LORA_EXPAND_CTAS_PER_SM >= 2 ? 113 : 225) * 1024;
+  P.base_stages = 2;
+  while (P.base_stages < 8 && total(P.base_stages + 1) <= cap) ++P.base_stages;
+  if (total(P.base_stages) > 225 * 1024) return LORA_ERR_UNSUPPORTED;
+  size_t smem = total(P.base_stages);
   if (smem < 80 * 1024) smem = 80 * 1024;  // at most two CTAs (2 x 256 TMEM columns) per SM
 
   const int64_t n_tot = a.slices.off[a.S] - a.slices.off[0];
@@ -327,9 +338,8 @@ lora_status expand_tc(const lora::ExpandArgs& a, lora_dtype dt, const Grouping& 
     return LORA_ERR_CUDA;
 
   const long slots = lora::num_piece_slots(a.tok, P.nvseg, lora::kExBM);
-  const long est = (a.tok + lora::kExBM - 1) / lora::kExBM + (P.vseg_indptr ? a.L : a.nseg) / 2;
-  const long target = 2L * dev.sms;
-  long tpc = (est * tiles + target - 1) / target;
+  const long target = static_cast<long>(LORA_EXPAND_CTAS_PER_SM) * dev.sms * LORA_EXPAND_WAVES;
+  long tpc = (slots * tiles + target - 1) / target;
   if (tpc < 1) tpc = 1;
   if (tpc > tiles) tpc = tiles;
   P.tiles_per_cta = static_cast<int>(tpc);

@@ -81,10 +81,17 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
   const uint32_t empty0 = full0 + 8 * P.stages;
   const uint32_t done_bar = empty0 + 8 * P.stages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * P.stages + 1);
+  int64_t* xrow_tok = reinterpret_cast<int64_t*>(bars + 2 * P.stages + 2);  // [128] x row index
 
   const int kb0 = split * P.kb_per;
   const int nk = max(0, min(P.nkb, kb0 + P.kb_per) - kb0);
 
+  if (tid < kTcBM) {
+    const int m = tid;
+    int srow = pc.lo + (m < rows ? m : 0);
+    if (P.row_list) srow = clampi(__ldg(P.row_list + srow), 0, p.tok - 1);
+    xrow_tok[m] = p.permutation ? clampi(__ldg(p.permutation + srow), 0, p.tok - 1) : srow;
+  }
   if (tid == 0) {
     for (int s = 0; s < P.stages; ++s) {
       mbar_init(full0 + 8 * s, kTcBM + 1);
@@ -106,12 +113,8 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
 
   if (warp < 4) {
     // =========================== producer: gather x rows, TMA the A block
-    const int m = tid;  // row of the piece handled by this thread
-    const bool row_ok = m < rows;
-    int srow = pc.lo + (row_ok ? m : 0);
-    if (P.row_list) srow = clampi(__ldg(P.row_list + srow), 0, p.tok - 1);
-    const int t = p.permutation ? clampi(__ldg(p.permutation + srow), 0, p.tok - 1) : srow;
-    const uint16_t* xrow = p.x + static_cast<int64_t>(t) * p.ld_x;
+    // chunk u = j*128 + tid of a stage -> row u/8, 16-byte chunk u%8: every warp
+    // instruction reads 4 rows x 128 contiguous bytes
     const uint32_t a_bytes = P.npad * 128;
     const int lag = P.stages - 1;
     for (int i = 0; i < nk && ok; ++i) {
@@ -125,11 +128,14 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
         tma_load_2d(xs + x_bytes, &P.tmap_A, full0 + 8 * s, k0, adapter * p.S * p.rs);
       }
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int j = 0; j < 8; ++j) {
+        const int u = j * kTcBM + tid;
+        const int row = u >> 3, c = u & 7;
         const int k = k0 + 8 * c;
-        const bool in = row_ok && k < p.K;
-        const uint32_t dst = xs + m * 128 + ((c ^ (m & 7)) << 4);
-        cp_async_16(dst, in ? static_cast<const void*>(xrow + k) : static_cast<const void*>(p.x),
+        const bool in = row < rows && k < p.K;
+        const uint32_t dst = xs + row * 128 + ((c ^ (row & 7)) << 4);
+        cp_async_16(dst, in ? static_cast<const void*>(p.x + xrow_tok[row] * p.ld_x + k)
+                            : static_cast<const void*>(p.x),
                     in ? 16u : 0u);
       }
       cp_async_commit();

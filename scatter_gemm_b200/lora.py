@@ -16,7 +16,8 @@ from typing import Optional, Sequence
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "liblora_sgmv.so")
+# LORA_SGMV_LIB may point at another build of the library (e.g. an installed copy)
+LIB_PATH = os.environ.get("LORA_SGMV_LIB") or os.path.join(_HERE, "liblora_sgmv.so")
 
 LORA_OK, LORA_ERR_INVALID_ARGUMENT, LORA_ERR_UNSUPPORTED, LORA_ERR_CUDA, LORA_ERR_BAD_VALUES = \
     range(5)
