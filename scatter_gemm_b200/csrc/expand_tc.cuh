@@ -11,19 +11,21 @@
 // This is the expand and the "scatter epilogue" of the sgl-kernel-xpu page
 // ("Decode LoRA kernels are optimized", section "Summary"), rebuilt for B200.
 //
-// Warp roles (192 threads):
+// Warp roles (288 threads):
 //   warp 0      TMEM allocation; lane 0 loads B tiles by TMA (the tensor map's
 //               inner extent is r, so the storage padding j >= r reads as zero)
 //               and issues the MMAs;
-//   warps 1-4   epilogue: one accumulator row per thread (TMEM lane = row),
-//               read-modify-write of the staged base row in shared memory;
-//   warp 5      data mover: the piece's rank activations once (cp.async,
-//               partial-size form zero-fills j >= r), then every base tile in
-//               both directions as one bulk async copy per row (256 bytes),
-//               loads running up to `base_stages - 1` tiles ahead and each
-//               stage refilled as soon as its stores have read it.
-// Staged base rows sit at a 272-byte pitch, so the row-per-thread phase
-// (32 rows, same columns) and the bulk copies are both free of bank conflicts.
+//   warps 1-4   consumers: (a) one accumulator row per thread (TMEM lane = row)
+//               updates its staged base row in shared memory, (b) the four
+//               warps write the tile back with coalesced 16-byte stores;
+//   warps 5-8   producers: the piece's rank activations once (cp.async, whose
+//               partial-size form zero-fills the padding j >= r), then the base
+//               tiles with coalesced 16-byte cp.async (two 256-byte rows per
+//               warp instruction) into a ring of stages; completion reaches the
+//               consumers through cp.async.mbarrier.arrive, so producers never
+//               block on their own copies.
+// The 16-byte chunks of a staged row are XOR-swizzled by the row index, so the
+// row-per-thread phase and the coalesced phases are free of bank conflicts.
 #pragma once
 
 #include "common.cuh"
@@ -35,9 +37,8 @@ namespace lora {
 
 constexpr int kExBM = 128;      // rows per piece
 constexpr int kExBN = 128;      // columns per tile
-constexpr int kExThreads = 192;
-constexpr int kExPitch = kExBN * 2 + 16;           // bytes per staged base row
-constexpr int kExStageBytes = kExBM * kExPitch;    // one staged base tile
+constexpr int kExThreads = 288;
+constexpr int kExStageBytes = kExBM * kExBN * 2;  // one staged base tile (32 KB)
 
 struct ExpandTcParams {
   CUtensorMap tmap_B;  // 2-D [L*N_tot rows, r cols] (row stride rs), box {rpad, 128}
@@ -61,6 +62,10 @@ struct ExpandTcParams {
 // B tiles (rows of rpad*2 bytes, canonical UMMA swizzle)
 __device__ __forceinline__ int swz_chunk(int c, int m, int rpad) {
   return rpad == 64 ? (c ^ (m & 7)) : rpad == 32 ? (c ^ ((m >> 1) & 3)) : (c ^ ((m >> 2) & 1));
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
 template <class E>
@@ -89,7 +94,7 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
                                              ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t base_ring = sbase;
-  const uint32_t rin = base_ring + ((P.base_stages * kExStageBytes + 1023) & ~1023);
+  const uint32_t rin = base_ring + P.base_stages * kExStageBytes;
   const uint32_t bring = rin + p.S * P.rin_bytes;
   int* trow = reinterpret_cast<int*>(smem + (bring - sbase) + P.b_stages * P.btile_bytes);
   int* srow_of = trow + kExBM;
@@ -100,7 +105,7 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
   const uint32_t tempty0 = tfull0 + 16;
   const uint32_t rin_bar = tempty0 + 16;
   const uint32_t xfull0 = rin_bar + 8;                  // base tile landed
-  const uint32_t xready0 = xfull0 + 8 * P.base_stages;  // base tile updated
+  const uint32_t xempty0 = xfull0 + 8 * P.base_stages;  // base tile written back
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * P.b_stages + 5 +
                                                     2 * P.base_stages);
 
@@ -123,10 +128,10 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
       mbar_init(tfull0 + 8 * b, 1);
       mbar_init(tempty0 + 8 * b, kExBM);
     }
-    mbar_init(rin_bar, 32);
+    mbar_init(rin_bar, kExBM);
     for (int s = 0; s < P.base_stages; ++s) {
-      mbar_init(xfull0 + 8 * s, 1);
-      mbar_init(xready0 + 8 * s, kExBM);
+      mbar_init(xfull0 + 8 * s, kExBM);
+      mbar_init(xempty0 + 8 * s, kExBM);
     }
     fence_mbar_init();
     tma_prefetch_desc(&P.tmap_B);
@@ -195,85 +200,71 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
-    // =========================== data mover
-    // (1) rank activations of every slice, zero-filled beyond r (lane l: rows l + 32i)
+  } else if (warp >= 5) {
+    // =========================== producers (128 threads)
+    const int pt = tid - 5 * 32;
+    // (1) rank activations of every slice, zero-filled beyond r (thread = row)
     {
+      const int m = pt;
+      const bool row_ok = m < rows;
+      const uint16_t* src0 = p.in_r + static_cast<int64_t>(srow_of[m]) * p.ld_in;
       const int nchunk = P.rpad / 8;
-      for (int i = 0; i < kExBM / 32; ++i) {
-        const int m = lane + 32 * i;
-        const bool row_ok = m < rows;
-        const uint16_t* src0 = p.in_r + static_cast<int64_t>(srow_of[m]) * p.ld_in;
-        for (int q = 0; q < p.S; ++q) {
-          for (int c = 0; c < nchunk; ++c) {
-            const int left = p.r - 8 * c;
-            const uint32_t nb = row_ok ? static_cast<uint32_t>(max(0, min(left, 8)) * 2) : 0u;
-            const uint32_t dst = rin + q * P.rin_bytes + m * (P.rpad * 2) +
-                                 (swz_chunk(c, m, P.rpad) << 4);
-            cp_async_16(dst, nb ? static_cast<const void*>(src0 + q * p.rs + 8 * c)
-                                : static_cast<const void*>(p.in_r), nb);
-          }
+      for (int q = 0; q < p.S; ++q) {
+        for (int c = 0; c < nchunk; ++c) {
+          const int left = p.r - 8 * c;
+          const uint32_t nb = row_ok ? static_cast<uint32_t>(max(0, min(left, 8)) * 2) : 0u;
+          const uint32_t dst = rin + q * P.rin_bytes + m * (P.rpad * 2) +
+                               (swz_chunk(c, m, P.rpad) << 4);
+          cp_async_16(dst, nb ? static_cast<const void*>(src0 + q * p.rs + 8 * c)
+                              : static_cast<const void*>(p.in_r), nb);
         }
       }
       cp_async_commit();
       cp_async_wait<0>();
-      fence_proxy_async_smem();
+      fence_proxy_async_smem();  // read by the MMA through the async proxy
       mbar_arrive(rin_bar);
     }
-    // (2) base tiles: one bulk copy per row and direction
-    auto row_bytes = [&](int t) {
-      int q, c0;
-      tile_info(t, q, c0);
-      return static_cast<uint32_t>(min(kExBN, p.slices.off[q + 1] - c0) * 2);
-    };
-    auto load_tile = [&](int t) {
-      int q, c0;
-      tile_info(t, q, c0);
-      const uint32_t nb = row_bytes(t);
-      const int s = t % P.base_stages;
-      const uint32_t stage = base_ring + s * kExStageBytes;
-      if (lane == 0) mbar_arrive_expect_tx(xfull0 + 8 * s, nb * rows);
-      __syncwarp();
-      for (int m = lane; m < rows; m += 32)
-        bulk_load(stage + m * kExPitch,
-                  p.base + static_cast<int64_t>(trow[m]) * p.ld_base + c0, nb, xfull0 + 8 * s);
-    };
-    const int pre = min(P.base_stages, ntl);
-    for (int t = 0; t < pre; ++t) load_tile(t);
+    // (2) base tiles: chunk u = j*128 + pt -> row u/16, logical chunk u%16
     for (int t = 0; t < ntl && ok; ++t) {
       const int s = t % P.base_stages;
-      ok = mbar_wait(xready0 + 8 * s, (t / P.base_stages) & 1);
-      ok = __all_sync(0xffffffffu, ok);
+      if (t >= P.base_stages) ok = mbar_wait(xempty0 + 8 * s, ((t / P.base_stages) - 1) & 1);
       if (!ok) break;
       int q, c0;
       tile_info(t, q, c0);
-      const uint32_t nb = row_bytes(t);
+      const int cend = p.slices.off[q + 1];
       const uint32_t stage = base_ring + s * kExStageBytes;
-      for (int m = lane; m < rows; m += 32)
-        bulk_store(p.base + static_cast<int64_t>(trow[m]) * p.ld_base + c0,
-                   stage + m * kExPitch, nb);
-      bulk_commit();
-      // refill the stage of tile t-1 once its stores have read shared memory
-      const int tn = t - 1 + P.base_stages;
-      if (t >= 1 && tn < ntl) {
-        bulk_wait_read<1>();
-        __syncwarp();
-        load_tile(tn);
+#pragma unroll 4
+      for (int j = 0; j < 16; ++j) {
+        const int u = j * kExBM + pt;
+        const int row = u >> 4, c = u & 15;
+        const int col = c0 + 8 * c;
+        const bool in = row < rows && col < cend;
+        cp_async_16(stage + row * 256 + ((c ^ (row & 15)) << 4),
+                    in ? static_cast<const void*>(p.base +
+                                                  static_cast<int64_t>(trow[row]) * p.ld_base +
+                                                  col)
+                       : static_cast<const void*>(p.base),
+                    in ? 16u : 0u);
       }
+      cp_async_arrive_noinc(xfull0 + 8 * s);
     }
-    bulk_wait_all();
+    cp_async_wait<0>();
   } else {
-    // =========================== epilogue (warps 1-4, one accumulator row per thread)
+    // =========================== consumers (warps 1-4)
     const int quarter = warp & 3;
-    const int m = quarter * 32 + lane;
+    const int m = quarter * 32 + lane;  // accumulator row of this thread
+    const int ct = tid - 32;            // 0..127 for the coalesced phase
     for (int t = 0; t < ntl; ++t) {
       const int s = t % P.base_stages, buf = t & 1;
       if (ok) ok = mbar_wait(xfull0 + 8 * s, (t / P.base_stages) & 1);
       if (ok) ok = mbar_wait(tfull0 + 8 * buf, (t >> 1) & 1);
       ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
       tc_fence_after();
-      uint8_t* rowp = smem + (base_ring - sbase) + s * kExStageBytes + m * kExPitch;
+      int q, c0;
+      tile_info(t, q, c0);
+      uint8_t* stage_p = smem + (base_ring - sbase) + s * kExStageBytes;
       const uint32_t tacc = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * kExBN;
+      // (a) row-per-thread: base + scaling * acc, in place in shared memory
 #pragma unroll 1
       for (int cc = 0; cc < kExBN / 16; ++cc) {
         float v[16];
@@ -282,10 +273,11 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
           tmem_ld_wait();
         }
         if (ok && m < rows) {
-          uint4* ptr = reinterpret_cast<uint4*>(rowp + cc * 32);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            uint4 w = ptr[h];
+            const int c = 2 * cc + h;
+            uint4* ptr = reinterpret_cast<uint4*>(stage_p + m * 256 + ((c ^ (m & 15)) << 4));
+            uint4 w = *ptr;
             uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -293,14 +285,30 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
               wv[e] = E::f2_to_u32(fmaf(scale, v[8 * h + 2 * e], b.x),
                                    fmaf(scale, v[8 * h + 2 * e + 1], b.y));
             }
-            ptr[h] = w;
+            *ptr = w;
           }
         }
       }
       tc_fence_before();
       mbar_arrive(tempty0 + 8 * buf);
-      fence_proxy_async_smem();  // the bulk store reads these rows through the async proxy
-      mbar_arrive(xready0 + 8 * s);
+      named_bar_sync(1, kExBM);  // every row of the tile is updated
+      // (b) coalesced write-back: chunk u = j*128 + ct -> row u/16, chunk u%16
+      const int cend = p.slices.off[q + 1];
+      if (ok) {
+#pragma unroll 4
+        for (int j = 0; j < 16; ++j) {
+          const int u = j * kExBM + ct;
+          const int row = u >> 4, c = u & 15;
+          const int col = c0 + 8 * c;
+          if (row < rows && col < cend) {
+            const uint4 w = *reinterpret_cast<const uint4*>(stage_p + row * 256 +
+                                                            ((c ^ (row & 15)) << 4));
+            *reinterpret_cast<uint4*>(p.base + static_cast<int64_t>(trow[row]) * p.ld_base +
+                                      col) = w;
+          }
+        }
+      }
+      mbar_arrive(xempty0 + 8 * s);  // the stage's shared memory may be refilled
     }
   }
 

@@ -31,7 +31,7 @@
 
 // Tuning constants of the expand (compile-time; defaults below).
 #ifndef LORA_EXPAND_CTAS_PER_SM
-#define LORA_EXPAND_CTAS_PER_SM 2   // 2: <= 113 KB shared memory per CTA; 1: deeper ring
+#define LORA_EXPAND_CTAS_PER_SM 2   // 2: <= 113 KB per CTA; 1: deep ring (<= 225 KB)
 #endif
 #ifndef LORA_EXPAND_WAVES
 #define LORA_EXPAND_WAVES 1         // resident-CTA waves the grid is sized for
