@@ -163,6 +163,39 @@ LORA_API lora_status lora_validate(const int32_t* seg_indptr, const int32_t* wei
 
 LORA_API size_t lora_validate_workspace_size(int tok);
 
+/* lora_shrink_static_scratch -- lora_shrink for callers that cannot allocate.
+ *
+ * The pages have no counterpart of this call.  Some callers of this library
+ * are handed only input and output buffers by a host framework (a custom-op or
+ * plugin interface of an inference engine) and have no allocator of their own:
+ * they cannot call cudaMalloc, which would bypass the framework's memory
+ * accounting and can synchronise the device, and they have no workspace to
+ * pass.  This entry point computes exactly what lora_shrink computes, with the
+ * same arguments minus the workspace, and allocates nothing: the scratch of the
+ * adapter-grouped schedule lives in a fixed array of LORA_STATIC_SCRATCH_BYTES
+ * (1 MiB) compiled into the library, which every GPU that loads the library
+ * holds until the process exits.
+ *
+ *  - Limit: lora_workspace_size(tok, nseg, L) must not exceed
+ *    LORA_STATIC_SCRATCH_BYTES (about tok + nseg + L <= 262,000); larger
+ *    problems return LORA_ERR_UNSUPPORTED before anything is enqueued.
+ *  - The first call on each device looks up the array's device address with
+ *    that device current (a CUDA runtime query, no allocation) and caches it;
+ *    make that first call before any stream capture.
+ *  - Every call on a device shares the one array and leaves its contents
+ *    behind; nothing in it has to start at zero.  Calls whose kernels overlap
+ *    on the GPU (e.g. on two streams) race on the array: serialise them.
+ * Returns as lora_shrink.
+ */
+#define LORA_STATIC_SCRATCH_BYTES (1u << 20)
+LORA_API lora_status lora_shrink_static_scratch(const void* x, int64_t ld_x, const void* A_stack,
+                                                const int32_t* seg_indptr,
+                                                const int32_t* weight_indices,
+                                                const int32_t* permutation, void* out_r,
+                                                int64_t ld_out, int tok, int K, int S, int r,
+                                                int rs, int nseg, int L, lora_dtype dtype,
+                                                void* stream);
+
 /* Kernel path (LORA_PATH_* bits) chosen by the last lora_shrink / lora_expand
  * call made on this host thread; 0 if none launched a kernel. */
 LORA_API int lora_last_path(void);

@@ -521,3 +521,57 @@ lora_status lora_validate(const int32_t* seg_indptr, const int32_t* weight_indic
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ scratch-free shrink
+//
+// lora_shrink_static_scratch serves callers that are handed only input and
+// output buffers and have no way to obtain device memory of their own.  Its
+// scratch (the row lists of the adapter-grouped schedule) lives in the
+// file-scope array below instead of a caller workspace.  Every GPU that loads
+// the library keeps this array until the process exits.
+
+static __device__ __align__(256) int32_t
+    g_lora_static_scratch[LORA_STATIC_SCRATCH_BYTES / sizeof(int32_t)];
+
+namespace {
+
+struct StaticScratchAddr {
+  std::atomic<int> ready{0};
+  void* ptr = nullptr;
+};
+StaticScratchAddr g_static_scratch_addr[kMaxDevices];
+std::mutex g_static_scratch_mu;
+
+// Device address of the static scratch on the current device.  The host-side
+// name of the array is only a stand-in, so the address is looked up once per
+// device, with that device current, and cached.  Null on failure.
+void* static_scratch_on_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  StaticScratchAddr& s = g_static_scratch_addr[dev];
+  if (s.ready.load(std::memory_order_acquire)) return s.ptr;
+  std::lock_guard<std::mutex> lk(g_static_scratch_mu);
+  if (!s.ready.load(std::memory_order_relaxed)) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_lora_static_scratch) != cudaSuccess || p == nullptr)
+      return nullptr;
+    s.ptr = p;
+    s.ready.store(1, std::memory_order_release);
+  }
+  return s.ptr;
+}
+
+}  // namespace
+
+extern "C" lora_status lora_shrink_static_scratch(
+    const void* x, int64_t ld_x, const void* A_stack, const int32_t* seg_indptr,
+    const int32_t* weight_indices, const int32_t* permutation, void* out_r, int64_t ld_out,
+    int tok, int K, int S, int r, int rs, int nseg, int L, lora_dtype dtype, void* stream) {
+  // the grouping pass writes every word of the scratch it later reads, so
+  // nothing has to be cleared between calls
+  if (lora_workspace_size(tok, nseg, L) > LORA_STATIC_SCRATCH_BYTES) return LORA_ERR_UNSUPPORTED;
+  void* ws = static_scratch_on_current_device();
+  if (ws == nullptr) return LORA_ERR_CUDA;
+  return lora_shrink(x, ld_x, A_stack, seg_indptr, weight_indices, permutation, out_r, ld_out,
+                     tok, K, S, r, rs, nseg, L, dtype, ws, LORA_STATIC_SCRATCH_BYTES, stream);
+}

@@ -265,3 +265,40 @@ def lora_validate(seg_indptr: torch.Tensor, weight_indices: torch.Tensor,
         raise LoraError("lora_validate", st)
     (torch.cuda.current_stream() if stream is None else stream).synchronize()
     return int(result.item())
+
+
+STATIC_SCRATCH_BYTES = 1 << 20
+
+
+def lora_shrink_static_scratch(x: torch.Tensor, A_stack: torch.Tensor, seg_indptr: torch.Tensor,
+                               weight_indices: torch.Tensor, permutation: Optional[torch.Tensor],
+                               out_r: torch.Tensor, *, num_slices: int,
+                               rank: Optional[int] = None, stream=None) -> torch.Tensor:
+    """lora_shrink for callers that cannot allocate device memory.
+
+    Same arguments and result as :func:`lora_shrink` without a workspace: the
+    library's own fixed 1 MiB device array holds the scratch.  Calls that
+    overlap on the GPU race on that array, and problems whose workspace would
+    exceed it raise LoraError (LORA_ERR_UNSUPPORTED)."""
+    l = lib()
+    f = l.lora_shrink_static_scratch
+    f.argtypes = [_P, _L, _P, _P, _P, _P, _P, _L] + [_I] * 8 + [_P]
+    f.restype = _I
+    dt = _dtype_code(x)
+    if A_stack.dtype != x.dtype or out_r.dtype != x.dtype:
+        raise TypeError("x, A_stack and out_r must share one element type")
+    if A_stack.dim() != 3 or not A_stack.is_contiguous():
+        raise ValueError("A_stack must be a contiguous [L, S*rs, K] tensor")
+    S = int(num_slices)
+    L, srs, K = A_stack.shape
+    rs = srs // S
+    r = rs if rank is None else int(rank)
+    tok = x.shape[0]
+    st = f(x.data_ptr(), _row_major(x, "x"), A_stack.data_ptr(),
+           _table(seg_indptr, "seg_indptr"), _table(weight_indices, "weight_indices"),
+           _table(permutation, "permutation", True), out_r.data_ptr(),
+           _row_major(out_r, "out_r"), tok, K, S, r, rs, seg_indptr.numel() - 1, L, dt,
+           _stream(stream))
+    if st != LORA_OK:
+        raise LoraError("lora_shrink_static_scratch", st)
+    return out_r
