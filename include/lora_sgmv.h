@@ -163,6 +163,61 @@ LORA_API lora_status lora_validate(const int32_t* seg_indptr, const int32_t* wei
 
 LORA_API size_t lora_validate_workspace_size(int tok);
 
+/* ---- identity-permutation variants --------------------------------------
+ * The other LoRA ops of the sgl-kernel-xpu page's file table (SGEMMLoraAFwd,
+ * SGEMMLoraBFwd, QKVLoraBFwd, GateUpLoraBFwd, EmbeddingLoraAFwd) take segments
+ * in token order: row i of every tensor belongs to token i.  The first four are
+ * lora_shrink / lora_expand with permutation = NULL and a fixed slice layout;
+ * arguments, errors and results are those of the call they forward to.
+ */
+
+/* lora_sgemm_a: out[i, q*rs + j] = sum_k x[i, k] * A_stack[a, q*rs + j, k]. */
+LORA_API lora_status lora_sgemm_a(const void* x, int64_t ld_x, const void* A_stack,
+                                  const int32_t* seg_indptr, const int32_t* weight_indices,
+                                  void* out, int64_t ld_out, int tok, int K, int S, int r,
+                                  int rs, int nseg, int L, lora_dtype dtype, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/* lora_sgemm_b: one slice of width N at column 0:
+ * base_out[i, c] += scalings[a] * sum_j in_r[i, j] * B_stack[a, c, j]   (B_stack [L, N, rs]). */
+LORA_API lora_status lora_sgemm_b(const void* in_r, int64_t ld_in, const void* B_stack,
+                                  const int32_t* seg_indptr, const int32_t* weight_indices,
+                                  const float* scalings, void* base_out, int64_t ld_base,
+                                  int tok, int N, int r, int rs, int nseg, int L,
+                                  lora_dtype dtype, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/* lora_qkv_b: three slices (q, k, v) at the HOST column offsets qkv_offsets[0..3]. */
+LORA_API lora_status lora_qkv_b(const void* in_r, int64_t ld_in, const void* B_stack,
+                                const int32_t* seg_indptr, const int32_t* weight_indices,
+                                const int32_t* qkv_offsets, const float* scalings,
+                                void* base_out, int64_t ld_base, int tok, int r, int rs,
+                                int nseg, int L, lora_dtype dtype, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/* lora_gate_up_b: two slices (gate, up) of width N each, at columns 0 and N. */
+LORA_API lora_status lora_gate_up_b(const void* in_r, int64_t ld_in, const void* B_stack,
+                                    const int32_t* seg_indptr, const int32_t* weight_indices,
+                                    const float* scalings, void* base_out, int64_t ld_base,
+                                    int tok, int N, int r, int rs, int nseg, int L,
+                                    lora_dtype dtype, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
+/* lora_embedding_a: LoRA A of an embedding layer.  The input row of a token is
+ * the one-hot vector of its id, so
+ *   out[i, j] = A_emb[a, j, ids[i]]   (j < r)
+ * for every segment s, a = weight_indices[s], i in its rows.
+ *   ids     [tok]        device int32 token ids in [0, V) (out-of-range ids are clamped)
+ *   A_emb   [L, rs, V]   device, vocabulary contiguous
+ *   out     [tok, ld_out] device, ld_out >= rs; only the valid columns j < r of rows in
+ *                        segments are written
+ * The grid bound ceil(tok/128) + nseg is known on the host, so no maximum
+ * segment length is needed and nothing is read back from the device. */
+LORA_API lora_status lora_embedding_a(const int32_t* ids, const void* A_emb,
+                                      const int32_t* seg_indptr, const int32_t* weight_indices,
+                                      void* out, int64_t ld_out, int tok, int V, int r, int rs,
+                                      int nseg, int L, lora_dtype dtype, void* stream);
+
 /* lora_shrink_static_scratch -- lora_shrink for callers that cannot allocate.
  *
  * The pages have no counterpart of this call.  Some callers of this library

@@ -43,6 +43,8 @@ def lib():
             l.oracle_encode.restype = ctypes.c_uint16
             l.oracle_encode_f64.argtypes = [ctypes.c_double, _I]
             l.oracle_encode_f64.restype = ctypes.c_uint16
+            l.oracle_embedding_a.argtypes = [_P, _P, _P, _P, _P, _L] + [_I] * 6
+            l.oracle_embedding_a.restype = _I
             l.oracle_set_threads.argtypes = [_I]
             l.oracle_set_threads.restype = None
             l.oracle_max_threads.argtypes = []
@@ -94,6 +96,17 @@ def expand(in_r, ld_in, B, seg_indptr, weight_indices, permutation, slice_offset
     return lib().oracle_expand(_ptr(in_r), ld_in, _ptr(B), _ptr(si), _ptr(wi), _ptr(pm),
                                _ptr(so), _ptr(sc), _ptr(base_out), ld_base, tok, S, r, rs,
                                nseg, L, _dt(dtype), mode)
+
+
+def embedding_a(ids, A_emb, seg_indptr, weight_indices, out, ld_out, tok, V, r, rs, nseg,
+                L) -> int:
+    """out (uint16 [tok, ld_out]) is modified in place."""
+    assert out.dtype == np.uint16 and out.flags.c_contiguous
+    ids = _c(ids, np.int32)
+    A_emb = _c(A_emb, np.uint16)
+    si, wi = _c(seg_indptr, np.int32), _c(weight_indices, np.int32)
+    return lib().oracle_embedding_a(_ptr(ids), _ptr(A_emb), _ptr(si), _ptr(wi), _ptr(out),
+                                    ld_out, tok, V, r, rs, nseg, L)
 
 
 # ---------------------------------------------------------------- problem helpers

@@ -210,6 +210,32 @@ int oracle_expand(const void* in_r, int64_t ld_in, const uint16_t* B_stack,
   return 0;
 }
 
+/* ---------------------------------------------------------------- embedding A */
+
+/* The embedding variant of the shrink (sgl-kernel-xpu page, file table:
+ * EmbeddingLoraAFwd): the "x" row of a token is the one-hot vector of its id,
+ * so the product with A selects one column of the adapter's A. */
+int oracle_embedding_a(const int32_t* ids, const uint16_t* A_emb, const int32_t* seg_indptr,
+                       const int32_t* weight_indices, uint16_t* out, int64_t ld_out,
+                       int tok, int V, int r, int rs, int nseg, int L) {
+  if (V < 1 || r < 1 || rs < r || ld_out < rs || tok < 0 || nseg < 0 || L < 1)
+    return ORACLE_BAD_DIMS;
+  for (int s = 0; s <= nseg; ++s)
+    if (seg_indptr[s] < 0 || seg_indptr[s] > tok || (s > 0 && seg_indptr[s] < seg_indptr[s - 1]))
+      return ORACLE_BAD_INDPTR;
+  for (int s = 0; s < nseg; ++s) {
+    const int a = weight_indices[s];
+    if (a < 0 || a >= L) return ORACLE_BAD_ADAPTER;
+    for (int i = seg_indptr[s]; i < seg_indptr[s + 1]; ++i) {
+      const int id = ids[i];
+      if (id < 0 || id >= V) return ORACLE_BAD_DIMS;
+      for (int j = 0; j < r; ++j)
+        out[(int64_t)i * ld_out + j] = A_emb[((int64_t)a * rs + j) * V + id];
+    }
+  }
+  return 0;
+}
+
 /* ---------------------------------------------------------------- threads */
 
 void oracle_set_threads(int n) { omp_set_num_threads(n > 0 ? n : 1); }

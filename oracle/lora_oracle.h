@@ -70,6 +70,14 @@ int oracle_expand(const void* in_r, int64_t ld_in, const uint16_t* B_stack,
                   int tok, int S, int r, int rs, int nseg, int L,
                   int dtype, int mode);
 
+/* out[i, j] = A_emb[a, j, ids[i]]  (j < r) for every segment s, a = weight_indices[s],
+ * i in [seg_indptr[s], seg_indptr[s+1]); rows are in token order (no permutation).
+ * A_emb is [L, rs, V] with the vocabulary dimension contiguous.  Returns
+ * ORACLE_BAD_DIMS for a token id outside [0, V). */
+int oracle_embedding_a(const int32_t* ids, const uint16_t* A_emb, const int32_t* seg_indptr,
+                       const int32_t* weight_indices, uint16_t* out, int64_t ld_out,
+                       int tok, int V, int r, int rs, int nseg, int L);
+
 /* element codec, exposed so the tests can pin it against other libraries */
 float oracle_decode(uint16_t h, int dtype);
 uint16_t oracle_encode(float f, int dtype);

@@ -35,10 +35,16 @@
 
 namespace lora {
 
-constexpr int kExBM = 128;      // rows per piece
-constexpr int kExBN = 128;      // columns per tile
+#ifndef LORA_EXPAND_BN
+#define LORA_EXPAND_BN 128  // columns per tile (128 or 256)
+#endif
+constexpr int kExBM = 128;               // rows per piece
+constexpr int kExBN = LORA_EXPAND_BN;    // columns per tile
+constexpr int kExCh = kExBN / 8;         // 16-byte chunks per staged row
+constexpr int kExTmemCols = 2 * kExBN;   // double-buffered accumulator
 constexpr int kExThreads = 288;
-constexpr int kExStageBytes = kExBM * kExBN * 2;  // one staged base tile (32 KB)
+constexpr int kExStageBytes = kExBM * kExBN * 2;  // one staged base tile
+static_assert(kExBN == 128 || kExBN == 256, "expand tile width");
 
 struct ExpandTcParams {
   CUtensorMap tmap_B;  // 2-D [L*N_tot rows, r cols] (row stride rs), box {rpad, 128}
@@ -80,13 +86,25 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
   const int t_begin = (blockIdx.x % ncg) * P.tiles_per_cta;
   const int ntl = min(P.tiles_total, t_begin + P.tiles_per_cta) - t_begin;
 
-  Piece pc;
+  if (ntl <= 0) return;
+  // Rows of a block slot start at slot*128: fetch their sorted rows and tokens
+  // while the tables are read.
+  const bool block_slot = slot < (p.tok + kExBM - 1) / kExBM;
+  int spec_srow = 0, spec_tok = 0;
+  if (tid < kExBM && block_slot) {
+    spec_srow = min(slot * kExBM + tid, p.tok - 1);
+    if (P.row_list) spec_srow = clampi(__ldg(P.row_list + spec_srow), 0, p.tok - 1);
+    spec_tok = p.permutation ? clampi(__ldg(p.permutation + spec_srow), 0, p.tok - 1)
+                             : spec_srow;
+  }
+  PieceInfo pc;
   const int32_t* indptr = P.vseg_indptr ? P.vseg_indptr : p.seg_indptr;
-  if (ntl <= 0 || !find_piece(indptr, P.nvseg, p.tok, kExBM, slot, pc)) return;
+  if (!find_piece_warp(indptr, P.vseg_indptr ? nullptr : p.weight_indices, p.scalings,
+                       P.nvseg, p.L, p.tok, kExBM, slot, pc))
+    return;
   const int rows = pc.hi - pc.lo;
-  const int adapter = P.vseg_indptr ? clampi(pc.seg, 0, p.L - 1)
-                                    : clampi(__ldg(p.weight_indices + pc.seg), 0, p.L - 1);
-  const float scale = __ldg(p.scalings + adapter);
+  const int adapter = pc.adapter;
+  const float scale = pc.per_adapter;
   if (scale == 0.f) return;  // zero scaling: the rows stay bit-identical
 
   // ---- shared memory: [base ring][rank activations S x][B ring][row tables][barriers]
@@ -114,10 +132,15 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
 
   if (tid < kExBM) {
     const int m = tid;
-    int sr = pc.lo + (m < rows ? m : 0);
-    if (P.row_list) sr = clampi(__ldg(P.row_list + sr), 0, p.tok - 1);
-    srow_of[m] = sr;
-    trow[m] = p.permutation ? clampi(__ldg(p.permutation + sr), 0, p.tok - 1) : sr;
+    if (block_slot) {
+      srow_of[m] = spec_srow;
+      trow[m] = spec_tok;
+    } else {
+      int sr = pc.lo + (m < rows ? m : 0);
+      if (P.row_list) sr = clampi(__ldg(P.row_list + sr), 0, p.tok - 1);
+      srow_of[m] = sr;
+      trow[m] = p.permutation ? clampi(__ldg(p.permutation + sr), 0, p.tok - 1) : sr;
+    }
   }
   if (tid == 0) {
     for (int s = 0; s < P.b_stages; ++s) {
@@ -137,7 +160,7 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
     tma_prefetch_desc(&P.tmap_B);
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_alloc(smem_u32(tmem_slot), kExTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -224,7 +247,7 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
       fence_proxy_async_smem();  // read by the MMA through the async proxy
       mbar_arrive(rin_bar);
     }
-    // (2) base tiles: chunk u = j*128 + pt -> row u/16, logical chunk u%16
+    // (2) base tiles: chunk u = j*128 + pt -> row u / kExCh, logical chunk u % kExCh
     for (int t = 0; t < ntl && ok; ++t) {
       const int s = t % P.base_stages;
       if (t >= P.base_stages) ok = mbar_wait(xempty0 + 8 * s, ((t / P.base_stages) - 1) & 1);
@@ -234,12 +257,12 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
       const int cend = p.slices.off[q + 1];
       const uint32_t stage = base_ring + s * kExStageBytes;
 #pragma unroll 4
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < kExCh; ++j) {
         const int u = j * kExBM + pt;
-        const int row = u >> 4, c = u & 15;
+        const int row = u / kExCh, c = u % kExCh;
         const int col = c0 + 8 * c;
         const bool in = row < rows && col < cend;
-        cp_async_16(stage + row * 256 + ((c ^ (row & 15)) << 4),
+        cp_async_16(stage + row * (kExBN * 2) + ((c ^ (row & (kExCh - 1))) << 4),
                     in ? static_cast<const void*>(p.base +
                                                   static_cast<int64_t>(trow[row]) * p.ld_base +
                                                   col)
@@ -276,7 +299,8 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int c = 2 * cc + h;
-            uint4* ptr = reinterpret_cast<uint4*>(stage_p + m * 256 + ((c ^ (m & 15)) << 4));
+            uint4* ptr = reinterpret_cast<uint4*>(stage_p + m * (kExBN * 2) +
+                                                  ((c ^ (m & (kExCh - 1))) << 4));
             uint4 w = *ptr;
             uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
@@ -292,17 +316,17 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
       tc_fence_before();
       mbar_arrive(tempty0 + 8 * buf);
       named_bar_sync(1, kExBM);  // every row of the tile is updated
-      // (b) coalesced write-back: chunk u = j*128 + ct -> row u/16, chunk u%16
+      // (b) coalesced write-back: chunk u = j*128 + ct -> row u / kExCh, chunk u % kExCh
       const int cend = p.slices.off[q + 1];
       if (ok) {
 #pragma unroll 4
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < kExCh; ++j) {
           const int u = j * kExBM + ct;
-          const int row = u >> 4, c = u & 15;
+          const int row = u / kExCh, c = u % kExCh;
           const int col = c0 + 8 * c;
           if (row < rows && col < cend) {
-            const uint4 w = *reinterpret_cast<const uint4*>(stage_p + row * 256 +
-                                                            ((c ^ (row & 15)) << 4));
+            const uint4 w = *reinterpret_cast<const uint4*>(stage_p + row * (kExBN * 2) +
+                                                            ((c ^ (row & (kExCh - 1))) << 4));
             *reinterpret_cast<uint4*>(p.base + static_cast<int64_t>(trow[row]) * p.ld_base +
                                       col) = w;
           }
@@ -315,7 +339,7 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, kExTmemCols);
   }
 }
 

@@ -22,6 +22,7 @@
 
 #include "../../include/lora_sgmv.h"
 #include "common.cuh"
+#include "embedding.cuh"
 #include "expand_tc.cuh"
 #include "general.cuh"
 #include "group.cuh"
@@ -35,6 +36,9 @@
 #endif
 #ifndef LORA_EXPAND_WAVES
 #define LORA_EXPAND_WAVES 1         // resident-CTA waves the grid is sized for
+#endif
+#ifndef LORA_SHRINK_CTAS_PER_SM
+#define LORA_SHRINK_CTAS_PER_SM 2  // 2: <= 110 KB shared memory per CTA; 1: deepest ring
 #endif
 #ifndef LORA_EXPAND_B_STAGES
 #define LORA_EXPAND_B_STAGES 3
@@ -67,12 +71,19 @@ struct DeviceFacts {
 DeviceFacts g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
+template <class E, int NSUB>
+void set_shrink_attrs() {
+  cudaFuncSetAttribute(lora::shrink_tc_kernel<E, NSUB>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  cudaFuncSetAttribute(lora::shrink_tc_kernel<E, NSUB>,
+                       cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+}
+
 template <class E>
 void set_kernel_attrs() {
-  cudaFuncSetAttribute(lora::shrink_tc_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       227 * 1024);
-  cudaFuncSetAttribute(lora::shrink_tc_kernel<E>,
-                       cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  set_shrink_attrs<E, 1>();
+  set_shrink_attrs<E, 2>();
+  set_shrink_attrs<E, 4>();
   cudaFuncSetAttribute(lora::expand_tc_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        227 * 1024);
   cudaFuncSetAttribute(lora::expand_general_kernel<E>,
@@ -105,7 +116,8 @@ const DeviceFacts* device_facts() {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int nclusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&nclusters, lora::shrink_tc_kernel<lora::Bf16>, &cfg) ==
+    if (cudaOccupancyMaxActiveClusters(&nclusters, lora::shrink_tc_kernel<lora::Bf16, 1>,
+                                       &cfg) ==
             cudaSuccess &&
         nclusters > 0)
       f.max_cluster = 16;
@@ -218,29 +230,39 @@ lora_status shrink_tc(const lora::ShrinkArgs& a, lora_dtype dt, const Grouping& 
   P.nvseg = g.vseg_indptr ? g.nvseg : a.nseg;
   P.npad = round_up(a.S * a.rs, 16);
   P.tmem_cols = P.npad <= 32 ? 32 : P.npad <= 64 ? 64 : P.npad <= 128 ? 128 : 256;
-  P.stage_bytes = lora::kTcBM * 128 + P.npad * 128;
-  const int budget = (P.npad <= 128 ? 110 : 200) * 1024;
+  // widest stage (64-K sub-tiles of x and A) that still leaves two stages, and
+  // room for the split-K partial, inside the shared-memory budget
+  const int budget = (LORA_SHRINK_CTAS_PER_SM >= 2 && P.npad <= 128 ? 110 : 220) * 1024;
+  const size_t part_bytes = sizeof(float) * lora::kTcBM * (P.npad + 1);
+  int nsub = lora::kTcMaxNSub;
+  for (;; nsub /= 2) {
+    const int sb = nsub * (lora::kTcBM * 128 + P.npad * 128);
+    if (nsub == 1 || (2 * sb <= budget - 2048 && static_cast<size_t>(2 * sb) >= part_bytes)) break;
+  }
+  P.stage_bytes = nsub * (lora::kTcBM * 128 + P.npad * 128);
   P.stages = (budget - 2048) / static_cast<int>(P.stage_bytes);
   P.stages = P.stages < 2 ? 2 : (P.stages > 8 ? 8 : P.stages);
-  const size_t part_bytes = sizeof(float) * lora::kTcBM * (P.npad + 1);
   while (static_cast<size_t>(P.stages) * P.stage_bytes < part_bytes) ++P.stages;
-  P.nkb = (a.K + lora::kTcBK - 1) / lora::kTcBK;
+  P.nkb = (a.K + nsub * lora::kTcAtomK - 1) / (nsub * lora::kTcAtomK);
 
   // K split over a cluster: the smallest power of two that gives every SM a CTA
-  // (expected pieces: one per 128 rows plus about half a piece per segment)
+  // (expected pieces: one per 128 rows plus about half a piece per segment),
+  // keeping at least four stages of K per CTA.  (Splitting further, to fill
+  // every resident CTA slot, measured slower: more partials to reduce.)
+  const size_t smem_need = static_cast<size_t>(P.stages) * P.stage_bytes + 1024 +
+                           8 * (2 * P.stages + 2) + 8 * lora::kTcBM + 16;
   const int est = (a.tok + lora::kTcBM - 1) / lora::kTcBM + (P.vseg_indptr ? a.L : a.nseg) / 2;
   int cs = 1;
-  while (cs < dev.max_cluster && est * cs < dev.sms && P.nkb >= 8 * cs) cs *= 2;
+  while (cs < dev.max_cluster && est * cs < dev.sms && P.nkb >= 4 * cs) cs *= 2;
   P.csplit = cs;
   P.kb_per = (P.nkb + cs - 1) / cs;
   P.idesc = lora::make_idesc_f16(dt == LORA_BF16 ? 1 : 0, lora::kTcBM, P.npad);
   if (!encode_2d(&P.tmap_A, dt, a.A, a.K, static_cast<uint64_t>(a.L) * a.S * a.rs,
-                 static_cast<uint64_t>(a.K) * 2, lora::kTcBK, P.npad,
+                 static_cast<uint64_t>(a.K) * 2, lora::kTcAtomK, P.npad,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return LORA_ERR_CUDA;
 
-  const size_t smem = static_cast<size_t>(P.stages) * P.stage_bytes + 1024 +
-                      8 * (2 * P.stages + 2) + 8 * lora::kTcBM + 16;
+  const size_t smem = smem_need;
   const long slots = lora::num_piece_slots(a.tok, P.nvseg, lora::kTcBM);
   cudaLaunchConfig_t cfg{};
   cudaLaunchAttribute attr[1];
@@ -256,7 +278,11 @@ lora_status shrink_tc(const lora::ShrinkArgs& a, lora_dtype dt, const Grouping& 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, lora::shrink_tc_kernel<E>, P);
+  if (smem > 227 * 1024) return LORA_ERR_UNSUPPORTED;
+  cudaError_t e;
+  if (nsub == 4) e = cudaLaunchKernelEx(&cfg, lora::shrink_tc_kernel<E, 4>, P);
+  else if (nsub == 2) e = cudaLaunchKernelEx(&cfg, lora::shrink_tc_kernel<E, 2>, P);
+  else e = cudaLaunchKernelEx(&cfg, lora::shrink_tc_kernel<E, 1>, P);
   ++g_launches;
   g_last_path = LORA_PATH_TENSOR | (cs > 1 ? LORA_PATH_SPLITK : 0) |
                 (P.vseg_indptr ? LORA_PATH_GROUPED : 0);
@@ -325,12 +351,16 @@ lora_status expand_tc(const lora::ExpandArgs& a, lora_dtype dt, const Grouping& 
     return ((static_cast<size_t>(bs) * lora::kExStageBytes + 1023) & ~size_t(1023)) + fixed +
            8 * (2 * P.b_stages + 5 + 2 * bs);
   };
-  const size_t cap = (LORA_EXPAND_CTAS_PER_SM >= 2 ? 113 : 225) * 1024;
+  // two CTAs per SM only when both accumulators fit twice in TMEM (512 columns)
+  const int ctas_per_sm = (LORA_EXPAND_CTAS_PER_SM >= 2 && lora::kExTmemCols <= 256) ? 2 : 1;
+  const size_t cap = (ctas_per_sm >= 2 ? 113 : 225) * 1024;
   P.base_stages = 2;
   while (P.base_stages < 8 && total(P.base_stages + 1) <= cap) ++P.base_stages;
   if (total(P.base_stages) > 225 * 1024) return LORA_ERR_UNSUPPORTED;
   size_t smem = total(P.base_stages);
-  if (smem < 80 * 1024) smem = 80 * 1024;  // at most two CTAs (2 x 256 TMEM columns) per SM
+  // keep the CTAs per SM within TMEM: 512 columns / kExTmemCols
+  const size_t min_smem = lora::kExTmemCols > 256 ? 116 * 1024 : 80 * 1024;
+  if (smem < min_smem) smem = min_smem;
 
   const int64_t n_tot = a.slices.off[a.S] - a.slices.off[0];
   if (!encode_2d(&P.tmap_B, dt, a.B, a.r, static_cast<uint64_t>(a.L) * n_tot,
@@ -338,7 +368,7 @@ lora_status expand_tc(const lora::ExpandArgs& a, lora_dtype dt, const Grouping& 
     return LORA_ERR_CUDA;
 
   const long slots = lora::num_piece_slots(a.tok, P.nvseg, lora::kExBM);
-  const long target = static_cast<long>(LORA_EXPAND_CTAS_PER_SM) * dev.sms * LORA_EXPAND_WAVES;
+  const long target = static_cast<long>(ctas_per_sm) * dev.sms * LORA_EXPAND_WAVES;
   long tpc = (slots * tiles + target - 1) / target;
   if (tpc < 1) tpc = 1;
   if (tpc > tiles) tpc = tiles;
@@ -521,6 +551,83 @@ lora_status lora_validate(const int32_t* seg_indptr, const int32_t* weight_indic
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ identity-permutation ops
+//
+// The other LoRA ops of the sgl-kernel-xpu page's file table (SGEMMLoraAFwd,
+// SGEMMLoraBFwd, QKVLoraBFwd, GateUpLoraBFwd, EmbeddingLoraAFwd) work on
+// segments in token order.  The first four are the shrink / expand with the
+// identity permutation and a fixed slice layout, so they forward to the same
+// kernels; the embedding one has a gather kernel of its own.
+
+extern "C" lora_status lora_sgemm_a(const void* x, int64_t ld_x, const void* A_stack,
+                                    const int32_t* seg_indptr, const int32_t* weight_indices,
+                                    void* out, int64_t ld_out, int tok, int K, int S, int r,
+                                    int rs, int nseg, int L, lora_dtype dtype, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  return lora_shrink(x, ld_x, A_stack, seg_indptr, weight_indices, nullptr, out, ld_out, tok, K,
+                     S, r, rs, nseg, L, dtype, workspace, workspace_bytes, stream);
+}
+
+extern "C" lora_status lora_sgemm_b(const void* in_r, int64_t ld_in, const void* B_stack,
+                                    const int32_t* seg_indptr, const int32_t* weight_indices,
+                                    const float* scalings, void* base_out, int64_t ld_base,
+                                    int tok, int N, int r, int rs, int nseg, int L,
+                                    lora_dtype dtype, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  if (N < 0) return LORA_ERR_INVALID_ARGUMENT;
+  const int32_t off[2] = {0, N};
+  return lora_expand(in_r, ld_in, B_stack, seg_indptr, weight_indices, nullptr, off, scalings,
+                     base_out, ld_base, tok, 1, r, rs, nseg, L, dtype, workspace,
+                     workspace_bytes, stream);
+}
+
+extern "C" lora_status lora_qkv_b(const void* in_r, int64_t ld_in, const void* B_stack,
+                                  const int32_t* seg_indptr, const int32_t* weight_indices,
+                                  const int32_t* qkv_offsets, const float* scalings,
+                                  void* base_out, int64_t ld_base, int tok, int r, int rs,
+                                  int nseg, int L, lora_dtype dtype, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  return lora_expand(in_r, ld_in, B_stack, seg_indptr, weight_indices, nullptr, qkv_offsets,
+                     scalings, base_out, ld_base, tok, 3, r, rs, nseg, L, dtype, workspace,
+                     workspace_bytes, stream);
+}
+
+extern "C" lora_status lora_gate_up_b(const void* in_r, int64_t ld_in, const void* B_stack,
+                                      const int32_t* seg_indptr, const int32_t* weight_indices,
+                                      const float* scalings, void* base_out, int64_t ld_base,
+                                      int tok, int N, int r, int rs, int nseg, int L,
+                                      lora_dtype dtype, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+  if (N < 0 || N > (1 << 30)) return LORA_ERR_INVALID_ARGUMENT;
+  const int32_t off[3] = {0, N, 2 * N};
+  return lora_expand(in_r, ld_in, B_stack, seg_indptr, weight_indices, nullptr, off, scalings,
+                     base_out, ld_base, tok, 2, r, rs, nseg, L, dtype, workspace,
+                     workspace_bytes, stream);
+}
+
+extern "C" lora_status lora_embedding_a(const int32_t* ids, const void* A_emb,
+                                        const int32_t* seg_indptr,
+                                        const int32_t* weight_indices, void* out,
+                                        int64_t ld_out, int tok, int V, int r, int rs, int nseg,
+                                        int L, lora_dtype dtype, void* stream) {
+  if (dtype != LORA_BF16 && dtype != LORA_FP16) return LORA_ERR_UNSUPPORTED;
+  if (tok < 0 || nseg < 0 || V < 1 || r < 1 || rs < r || L < 1 || ld_out < rs)
+    return LORA_ERR_INVALID_ARGUMENT;
+  if (tok == 0 || nseg == 0) return LORA_OK;
+  if (!ids || !A_emb || !seg_indptr || !weight_indices || !out) return LORA_ERR_INVALID_ARGUMENT;
+  if (!aligned_to(ids, 4) || !aligned_to(A_emb, 2) || !aligned_to(out, 2) ||
+      !aligned_to(seg_indptr, 4) || !aligned_to(weight_indices, 4))
+    return LORA_ERR_INVALID_ARGUMENT;
+  const long slots = lora::num_piece_slots(tok, nseg, lora::kEmbBM);
+  lora::embedding_a_kernel<<<static_cast<unsigned>(slots), 128, 0,
+                             static_cast<cudaStream_t>(stream)>>>(
+      ids, static_cast<const uint16_t*>(A_emb), seg_indptr, weight_indices,
+      static_cast<uint16_t*>(out), ld_out, tok, V, r, rs, nseg, L);
+  ++g_launches;
+  g_last_path = LORA_PATH_GENERAL;
+  return launch_status();
+}
 
 // ------------------------------------------------------------------ scratch-free shrink
 //

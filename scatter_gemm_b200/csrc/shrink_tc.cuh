@@ -10,9 +10,10 @@
 //
 //  - warps 0-3 gather the piece's x rows (row m = token perm[lo+m]) with
 //    16-byte cp.async straight into the 128-byte-swizzled K-major layout the
-//    MMA reads, K block by K block (64 elements), through a ring of stages;
-//  - thread 0 loads the adapter's A block of the stage with one TMA tiled
-//    copy (rows a*S*rs ... + NPAD, 64 K columns; out-of-range rows and K
+//    MMA reads, through a ring of stages of up to LORA_SHRINK_BK K elements
+//    (the host picks the widest that fits two stages; 64 measured best);
+//  - thread 0 loads the adapter's A block of the stage with TMA tiled copies
+//    (rows a*S*rs ... + NPAD, 64 K columns each; out-of-range rows and K
 //    columns are zero-filled by the TMA unit);
 //  - warp 4 issues the MMAs and returns each stage with tcgen05.commit;
 //  - warps 0-3 then read the accumulator back (tcgen05.ld, one row per
@@ -34,7 +35,12 @@
 namespace lora {
 
 constexpr int kTcBM = 128;   // rows per piece (MMA M)
-constexpr int kTcBK = 64;    // K elements per stage (one 128-byte swizzle row)
+constexpr int kTcAtomK = 64; // K elements of one 128-byte swizzle atom row
+#ifndef LORA_SHRINK_BK
+#define LORA_SHRINK_BK 64     // widest stage: K elements of every x row (64 = 128 bytes)
+#endif
+constexpr int kTcMaxNSub = LORA_SHRINK_BK / kTcAtomK;
+static_assert(kTcMaxNSub == 1 || kTcMaxNSub == 2 || kTcMaxNSub == 4, "stage K width");
 constexpr int kTcThreads = 160;
 
 struct ShrinkTcParams {
@@ -53,9 +59,12 @@ struct ShrinkTcParams {
   uint32_t stage_bytes;
 };
 
-template <class E>
+// NSUB: 64-K sub-tiles per stage (stage K width = 64 * NSUB)
+template <class E, int NSUB>
 __global__ void __launch_bounds__(kTcThreads, 1)
 shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
+  constexpr int kTcNSub = NSUB;
+  constexpr int kTcBK = NSUB * kTcAtomK;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const ShrinkArgs& p = P.a;
   const int tid = threadIdx.x;
@@ -63,19 +72,28 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
   const int split = blockIdx.x % P.csplit;
   const int slot = blockIdx.x / P.csplit;
 
-  // ---- piece of this cluster (identical in all its CTAs)
-  Piece pc;
+  // ---- piece of this cluster (identical in all its CTAs).  Rows of a block
+  // slot start at slot*128, so their tokens are fetched while the tables are read.
+  const bool block_slot = slot < (p.tok + kTcBM - 1) / kTcBM;
+  int spec_tok = 0;
+  if (tid < kTcBM && block_slot) {
+    int sr = min(slot * kTcBM + tid, p.tok - 1);
+    if (P.row_list) sr = clampi(__ldg(P.row_list + sr), 0, p.tok - 1);
+    spec_tok = p.permutation ? clampi(__ldg(p.permutation + sr), 0, p.tok - 1) : sr;
+  }
+  PieceInfo pc;
   const int32_t* indptr = P.vseg_indptr ? P.vseg_indptr : p.seg_indptr;
-  if (!find_piece(indptr, P.nvseg, p.tok, kTcBM, slot, pc)) return;
+  if (!find_piece_warp(indptr, P.vseg_indptr ? nullptr : p.weight_indices, nullptr, P.nvseg,
+                       p.L, p.tok, kTcBM, slot, pc))
+    return;
   const int rows = pc.hi - pc.lo;
-  const int adapter = P.vseg_indptr ? clampi(pc.seg, 0, p.L - 1)
-                                    : clampi(__ldg(p.weight_indices + pc.seg), 0, p.L - 1);
+  const int adapter = pc.adapter;
 
   // ---- shared memory carve-up (1024-aligned stages, then barriers)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t x_bytes = kTcBM * 128;
+  const uint32_t x_bytes = kTcNSub * kTcBM * 128;  // kTcNSub sub-tiles of 128 rows x 128 B
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.stages * P.stage_bytes);
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * P.stages;
@@ -88,9 +106,13 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
 
   if (tid < kTcBM) {
     const int m = tid;
-    int srow = pc.lo + (m < rows ? m : 0);
-    if (P.row_list) srow = clampi(__ldg(P.row_list + srow), 0, p.tok - 1);
-    xrow_tok[m] = p.permutation ? clampi(__ldg(p.permutation + srow), 0, p.tok - 1) : srow;
+    if (block_slot) {
+      xrow_tok[m] = spec_tok;
+    } else {
+      int srow = pc.lo + (m < rows ? m : 0);
+      if (P.row_list) srow = clampi(__ldg(P.row_list + srow), 0, p.tok - 1);
+      xrow_tok[m] = p.permutation ? clampi(__ldg(p.permutation + srow), 0, p.tok - 1) : srow;
+    }
   }
   if (tid == 0) {
     for (int s = 0; s < P.stages; ++s) {
@@ -115,7 +137,8 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
     // =========================== producer: gather x rows, TMA the A block
     // chunk u = j*128 + tid of a stage -> row u/8, 16-byte chunk u%8: every warp
     // instruction reads 4 rows x 128 contiguous bytes
-    const uint32_t a_bytes = P.npad * 128;
+    const uint32_t a_sub = P.npad * 128;  // one 64-K sub-tile of A
+    const uint32_t a_bytes = kTcNSub * a_sub;
     const int lag = P.stages - 1;
     for (int i = 0; i < nk && ok; ++i) {
       const int s = i % P.stages;
@@ -125,15 +148,21 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
       const int k0 = (kb0 + i) * kTcBK;
       if (tid == 0) {
         mbar_arrive_expect_tx(full0 + 8 * s, a_bytes);
-        tma_load_2d(xs + x_bytes, &P.tmap_A, full0 + 8 * s, k0, adapter * p.S * p.rs);
-      }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+        for (int sub = 0; sub < kTcNSub; ++sub)
+          tma_load_2d(xs + x_bytes + sub * a_sub, &P.tmap_A, full0 + 8 * s, k0 + sub * kTcAtomK,
+                      adapter * p.S * p.rs);
+      }
+      // chunk u = j*128 + tid -> row u / (BK/8), 16-byte chunk u % (BK/8): a warp
+      // instruction reads 512 / (BK/8 * 16 / 512) rows of contiguous bytes
+#pragma unroll 8
+      for (int j = 0; j < kTcBK / 8; ++j) {
         const int u = j * kTcBM + tid;
-        const int row = u >> 3, c = u & 7;
+        const int row = u / (kTcBK / 8), c = u % (kTcBK / 8);
         const int k = k0 + 8 * c;
         const bool in = row < rows && k < p.K;
-        const uint32_t dst = xs + row * 128 + ((c ^ (row & 7)) << 4);
+        const uint32_t dst = xs + (c >> 3) * (kTcBM * 128) + row * 128 +
+                             (((c & 7) ^ (row & 7)) << 4);
         cp_async_16(dst, in ? static_cast<const void*>(p.x + xrow_tok[row] * p.ld_x + k)
                             : static_cast<const void*>(p.x),
                     in ? 16u : 0u);
@@ -164,8 +193,9 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
         const uint32_t as = xs + x_bytes;
 #pragma unroll
         for (int kk = 0; kk < kTcBK / 16; ++kk) {
-          const uint64_t ad = make_sdesc(xs + kk * 32, 128, 2);
-          const uint64_t bd = make_sdesc(as + kk * 32, 128, 2);
+          const uint32_t sub = kk >> 2, k16 = kk & 3;
+          const uint64_t ad = make_sdesc(xs + sub * (kTcBM * 128) + k16 * 32, 128, 2);
+          const uint64_t bd = make_sdesc(as + sub * (P.npad * 128) + k16 * 32, 128, 2);
           tc_mma_f16(tmem, ad, bd, P.idesc, (i > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(empty0 + 8 * s);

@@ -302,3 +302,101 @@ def lora_shrink_static_scratch(x: torch.Tensor, A_stack: torch.Tensor, seg_indpt
     if st != LORA_OK:
         raise LoraError("lora_shrink_static_scratch", st)
     return out_r
+
+
+# ----------------------------------------------------------------------------
+# identity-permutation ops of the same page (segments in token order)
+# ----------------------------------------------------------------------------
+
+def _fn(name, argtypes):
+    f = getattr(lib(), name)
+    f.argtypes = argtypes
+    f.restype = _I
+    return f
+
+
+def _check(name, st):
+    if st != LORA_OK:
+        raise LoraError(name, st)
+
+
+def sgemm_lora_a_fwd(x, A_stack, seg_indptr, weight_indices, out, *, num_slices=1, rank=None,
+                     workspace=None, stream=None):
+    """out[i, q*rs+j] = sum_k x[i, k] * A_stack[a, q*rs+j, k] (no permutation)."""
+    L, srs, K = A_stack.shape
+    S = int(num_slices)
+    rs = srs // S
+    r = rs if rank is None else int(rank)
+    ws, wsb = _ws(workspace)
+    f = _fn("lora_sgemm_a", [_P, _L, _P, _P, _P, _P, _L] + [_I] * 8 + [_P, _Z, _P])
+    _check("lora_sgemm_a", f(x.data_ptr(), _row_major(x, "x"), A_stack.data_ptr(),
+                             _table(seg_indptr, "seg_indptr"),
+                             _table(weight_indices, "weight_indices"), out.data_ptr(),
+                             _row_major(out, "out"), x.shape[0], K, S, r, rs,
+                             seg_indptr.numel() - 1, L, _dtype_code(x), ws, wsb,
+                             _stream(stream)))
+    return out
+
+
+def _expand_like(name, in_r, B_stack, seg_indptr, weight_indices, scalings, base_out, rank,
+                 workspace, stream, extra_front=(), extra_types=(), n_arg=None):
+    L, n_tot, rs = B_stack.shape
+    r = rs if rank is None else int(rank)
+    ws, wsb = _ws(workspace)
+    types = [_P, _L, _P, _P, _P] + list(extra_types) + [_P, _P, _L, _I] + \
+        ([_I] if n_arg is not None else []) + [_I] * 5 + [_P, _Z, _P]
+    f = _fn(name, types)
+    args = [in_r.data_ptr(), _row_major(in_r, "in_r"), B_stack.data_ptr(),
+            _table(seg_indptr, "seg_indptr"), _table(weight_indices, "weight_indices")]
+    args += list(extra_front)
+    args += [scalings.data_ptr(), base_out.data_ptr(), _row_major(base_out, "base_out"),
+             base_out.shape[0]]
+    if n_arg is not None:
+        args.append(n_arg)
+    args += [r, rs, seg_indptr.numel() - 1, L, _dtype_code(base_out), ws, wsb, _stream(stream)]
+    _check(name, f(*args))
+    return base_out
+
+
+def sgemm_lora_b_fwd(in_r, B_stack, seg_indptr, weight_indices, scalings, base_out, *, rank=None,
+                     workspace=None, stream=None):
+    """base_out[i, c] += scalings[a] * sum_j in_r[i, j] * B_stack[a, c, j] (one slice)."""
+    return _expand_like("lora_sgemm_b", in_r, B_stack, seg_indptr, weight_indices, scalings,
+                        base_out, rank, workspace, stream, n_arg=B_stack.shape[1])
+
+
+def qkv_lora_b_fwd(in_r, B_stack, seg_indptr, weight_indices, qkv_offsets, scalings, base_out, *,
+                   rank=None, workspace=None, stream=None):
+    """Expand into three slices q, k, v at host column offsets qkv_offsets[0..3]."""
+    off = [int(v) for v in qkv_offsets]
+    if len(off) != 4:
+        raise ValueError("qkv_offsets needs 4 entries")
+    arr = (ctypes.c_int32 * 4)(*off)
+    return _expand_like("lora_qkv_b", in_r, B_stack, seg_indptr, weight_indices, scalings,
+                        base_out, rank, workspace, stream,
+                        extra_front=[ctypes.cast(arr, ctypes.c_void_p)], extra_types=[_P])
+
+
+def gate_up_lora_b_fwd(in_r, B_stack, seg_indptr, weight_indices, scalings, base_out, *,
+                       rank=None, workspace=None, stream=None):
+    """Expand into two equal slices (gate, up) at columns 0 and N."""
+    return _expand_like("lora_gate_up_b", in_r, B_stack, seg_indptr, weight_indices, scalings,
+                        base_out, rank, workspace, stream, n_arg=B_stack.shape[1] // 2)
+
+
+def embedding_lora_a_fwd(ids, A_emb, seg_indptr, weight_indices, out, *, rank=None, stream=None):
+    """out[i, j] = A_emb[a, j, ids[i]] for j < rank (A_emb [L, rs, V])."""
+    L, rs, V = A_emb.shape
+    r = rs if rank is None else int(rank)
+    f = _fn("lora_embedding_a", [_P, _P, _P, _P, _P, _L] + [_I] * 7 + [_P])
+    _check("lora_embedding_a", f(_table(ids, "ids"), A_emb.data_ptr(),
+                                 _table(seg_indptr, "seg_indptr"),
+                                 _table(weight_indices, "weight_indices"), out.data_ptr(),
+                                 _row_major(out, "out"), ids.numel(), V, r, rs,
+                                 seg_indptr.numel() - 1, L, _dtype_code(out), _stream(stream)))
+    return out
+
+
+# the chunked-SGMV pair under the names the pages use
+chunked_sgmv_lora_shrink_fwd = lora_shrink
+chunked_sgmv_lora_expand_fwd = lora_expand

@@ -433,3 +433,39 @@ def test_table_checks_flag_each_kind_of_bad_table():
 def test_nan_sentinels_are_nan():
     for dt, bits in NAN_BITS.items():
         assert np.isnan(from_bits(np.array([bits], dtype=np.uint16), dt)[0])
+
+
+# ----------------------------------------------------------------------------
+# embedding variant: the shrink of one-hot rows
+# ----------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_embedding_a_is_the_shrink_of_one_hot_rows(seed):
+    """With x_t = e_{id_t}, the shrink's out_r equals the embedding lookup (bit
+    exact: each sum has one nonzero term); identity permutation, one slice."""
+    rng = np.random.default_rng(seed)
+    V, r, rs, L, tok = 37, 5, 8, 3, 23
+    p = tiny_problem(seed, "bf16", tok=tok, K=V, slices=[8], r=r, rs=rs, L=L, nseg=4,
+                     ld_pad=0, col_lead=0)
+    p.permutation = np.arange(p.tok, dtype=np.int32)
+    ids = rng.integers(0, V, size=p.tok).astype(np.int32)
+    xf = np.zeros((p.tok, p.ld_x), dtype=np.float32)
+    xf[np.arange(p.tok), ids] = 1.0
+    via_shrink = oracle.shrink_problem(p, x=to_bits(xf, "bf16"))
+    A_emb = p.A.reshape(L, rs, V)  # [L, S*rs, K] with S = 1 and K = V
+    out = np.full((p.tok, rs), 0x7FFF, dtype=np.uint16)
+    assert oracle.embedding_a(ids, A_emb, p.seg_indptr, p.weight_indices, out, rs, p.tok, V, r,
+                              rs, p.nseg, L) == 0
+    assert np.array_equal(out, via_shrink)
+    # and directly: the adapter's column of the id
+    for s in range(p.nseg):
+        for i in range(p.seg_indptr[s], p.seg_indptr[s + 1]):
+            assert np.array_equal(out[i, :r], A_emb[p.weight_indices[s], :r, ids[i]])
+
+
+def test_embedding_a_rejects_out_of_vocabulary_ids():
+    A = np.zeros((1, 4, 10), dtype=np.uint16)
+    out = np.zeros((3, 4), dtype=np.uint16)
+    assert oracle.embedding_a(np.array([1, 10, 2]), A, np.array([0, 3]), np.array([0]), out, 4,
+                              3, 10, 4, 4, 1, 1) == oracle.BAD_DIMS
