@@ -33,6 +33,10 @@
 #include "sched.cuh"
 #include "sm100.cuh"
 
+#ifndef LORA_EXPAND_INTERLEAVE
+#define LORA_EXPAND_INTERLEAVE 1
+#endif
+
 namespace lora {
 
 #ifndef LORA_EXPAND_BN
@@ -83,8 +87,18 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
   const int warp = tid >> 5, lane = tid & 31;
   const int ncg = (P.tiles_total + P.tiles_per_cta - 1) / P.tiles_per_cta;
   const int slot = blockIdx.x / ncg;
-  const int t_begin = (blockIdx.x % ncg) * P.tiles_per_cta;
+  const int cg = blockIdx.x % ncg;
+#if LORA_EXPAND_INTERLEAVE
+  // column group cg takes tiles cg, cg+ncg, cg+2*ncg, ...: the CTAs of one piece
+  // (consecutive blocks, launched together) stream adjacent column tiles of the
+  // same rows at about the same time, so DRAM sees long runs of each row
+  const int ntl = cg < P.tiles_total ? (P.tiles_total - cg + ncg - 1) / ncg : 0;
+#define LORA_TILE(t) (cg + (t) * ncg)
+#else
+  const int t_begin = cg * P.tiles_per_cta;
   const int ntl = min(P.tiles_total, t_begin + P.tiles_per_cta) - t_begin;
+#define LORA_TILE(t) (t_begin + (t))
+#endif
 
   if (ntl <= 0) return;
   // Rows of a block slot start at slot*128: fetch their sorted rows and tokens
@@ -171,7 +185,7 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
 
   // tile t of this CTA -> (slice, first column)
   auto tile_info = [&](int t, int& q, int& c0) {
-    const int g = t_begin + t;
+    const int g = LORA_TILE(t);
     q = 0;
 #pragma unroll
     for (int k = 1; k < LORA_MAX_SLICES; ++k)
@@ -344,3 +358,5 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
 }
 
 }  // namespace lora
+
+#undef LORA_TILE

@@ -40,6 +40,9 @@
 #ifndef LORA_SHRINK_CTAS_PER_SM
 #define LORA_SHRINK_CTAS_PER_SM 2  // 2: <= 110 KB shared memory per CTA; 1: deepest ring
 #endif
+#ifndef LORA_SHRINK_MIN_SPLIT
+#define LORA_SHRINK_MIN_SPLIT 1    // smallest K split (CTAs per cluster) of the shrink
+#endif
 #ifndef LORA_EXPAND_B_STAGES
 #define LORA_EXPAND_B_STAGES 3
 #endif
@@ -253,7 +256,9 @@ lora_status shrink_tc(const lora::ShrinkArgs& a, lora_dtype dt, const Grouping& 
                            8 * (2 * P.stages + 2) + 8 * lora::kTcBM + 16;
   const int est = (a.tok + lora::kTcBM - 1) / lora::kTcBM + (P.vseg_indptr ? a.L : a.nseg) / 2;
   int cs = 1;
-  while (cs < dev.max_cluster && est * cs < dev.sms && P.nkb >= 4 * cs) cs *= 2;
+  while (cs < dev.max_cluster && P.nkb >= 4 * cs &&
+         (est * cs < dev.sms || cs < LORA_SHRINK_MIN_SPLIT))
+    cs *= 2;
   P.csplit = cs;
   P.kb_per = (P.nkb + cs - 1) / cs;
   P.idesc = lora::make_idesc_f16(dt == LORA_BF16 ? 1 : 0, lora::kTcBM, P.npad);

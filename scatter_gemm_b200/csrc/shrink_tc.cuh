@@ -32,6 +32,10 @@
 #include "sched.cuh"
 #include "sm100.cuh"
 
+#ifndef LORA_SHRINK_INTERLEAVE
+#define LORA_SHRINK_INTERLEAVE 1
+#endif
+
 namespace lora {
 
 constexpr int kTcBM = 128;   // rows per piece (MMA M)
@@ -101,8 +105,18 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * P.stages + 1);
   int64_t* xrow_tok = reinterpret_cast<int64_t*>(bars + 2 * P.stages + 2);  // [128] x row index
 
+  // K blocks of this CTA.  Interleaved over the cluster (CTA c takes blocks
+  // c, c+C, c+2C, ...), so the C co-scheduled CTAs of a piece read C adjacent
+  // 128-byte runs of every row at about the same time: DRAM sees contiguous
+  // C*128-byte pieces of each gathered row instead of scattered 128-byte ones.
+#if LORA_SHRINK_INTERLEAVE
+  const int nk = split < P.nkb ? (P.nkb - split + P.csplit - 1) / P.csplit : 0;
+#define LORA_KB(i) (split + (i) * P.csplit)
+#else
   const int kb0 = split * P.kb_per;
   const int nk = max(0, min(P.nkb, kb0 + P.kb_per) - kb0);
+#define LORA_KB(i) (kb0 + (i))
+#endif
 
   if (tid < kTcBM) {
     const int m = tid;
@@ -145,7 +159,7 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
       if (i >= P.stages) ok = mbar_wait(empty0 + 8 * s, ((i / P.stages) - 1) & 1);
       if (!ok) break;
       const uint32_t xs = sbase + s * P.stage_bytes;
-      const int k0 = (kb0 + i) * kTcBK;
+      const int k0 = LORA_KB(i) * kTcBK;
       if (tid == 0) {
         mbar_arrive_expect_tx(full0 + 8 * s, a_bytes);
 #pragma unroll
@@ -272,3 +286,5 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
 }
 
 }  // namespace lora
+
+#undef LORA_KB
