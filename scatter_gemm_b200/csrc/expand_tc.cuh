@@ -11,19 +11,20 @@
 // This is the expand and the "scatter epilogue" of the sgl-kernel-xpu page
 // ("Decode LoRA kernels are optimized", section "Summary"), rebuilt for B200.
 //
-// Warp roles (288 threads):
+// Warp roles (416 threads):
 //   warp 0      TMEM allocation; lane 0 loads B tiles by TMA (the tensor map's
 //               inner extent is r, so the storage padding j >= r reads as zero)
 //               and issues the MMAs;
-//   warps 1-4   consumers: (a) one accumulator row per thread (TMEM lane = row)
-//               updates its staged base row in shared memory, (b) the four
-//               warps write the tile back with coalesced 16-byte stores;
-//   warps 5-8   producers: the piece's rank activations once (cp.async, whose
-//               partial-size form zero-fills the padding j >= r), then the base
-//               tiles with coalesced 16-byte cp.async (two 256-byte rows per
-//               warp instruction) into a ring of stages; completion reaches the
-//               consumers through cp.async.mbarrier.arrive, so producers never
-//               block on their own copies.
+//   warps 1-8   consumers, two per TMEM lane quarter (one per half of the
+//               tile's columns): (a) one accumulator row per thread updates its
+//               staged base row in shared memory, (b) the eight warps write the
+//               tile back with coalesced 16-byte stores;
+//   warps 9-12  producers: the piece's rank activations (cp.async, whose
+//               partial-size form zero-fills the padding j >= r) overlapped
+//               with the first base tiles, then the base tiles with coalesced
+//               16-byte cp.async (two 256-byte rows per warp instruction) into a
+//               ring of stages; completion reaches the consumers through
+//               cp.async.mbarrier.arrive, so producers never block on a tile.
 // The 16-byte chunks of a staged row are XOR-swizzled by the row index, so the
 // row-per-thread phase and the coalesced phases are free of bank conflicts.
 #pragma once
@@ -42,12 +43,22 @@ namespace lora {
 #ifndef LORA_EXPAND_BN
 #define LORA_EXPAND_BN 128  // columns per tile (128 or 256)
 #endif
+#ifndef LORA_EXPAND_LD_BATCH
+#define LORA_EXPAND_LD_BATCH 2  // 16-column TMEM loads in flight per consumer thread
+#endif
+#ifndef LORA_EXPAND_MIN_BLOCKS
+#define LORA_EXPAND_MIN_BLOCKS 2  // co-resident CTAs per SM the register budget must allow
+#endif
 constexpr int kExBM = 128;               // rows per piece
 constexpr int kExBN = LORA_EXPAND_BN;    // columns per tile
 constexpr int kExCh = kExBN / 8;         // 16-byte chunks per staged row
 constexpr int kExTmemCols = 2 * kExBN;   // double-buffered accumulator
-constexpr int kExThreads = 288;
+constexpr int kExConsumers = 256;        // warps 1-8: two warps per TMEM lane quarter
+constexpr int kExProducers = 128;        // warps 9-12
+constexpr int kExThreads = 32 + kExConsumers + kExProducers;
 constexpr int kExStageBytes = kExBM * kExBN * 2;  // one staged base tile
+constexpr int kExLdBatch = LORA_EXPAND_LD_BATCH;   // TMEM chunks loaded per wait
+static_assert((kExBN / 32) % kExLdBatch == 0, "batch must divide a half tile");
 static_assert(kExBN == 128 || kExBN == 256, "expand tile width");
 
 struct ExpandTcParams {
@@ -79,7 +90,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
 }
 
 template <class E>
-__global__ void __launch_bounds__(kExThreads, 1)
+__global__ void __launch_bounds__(kExThreads, LORA_EXPAND_MIN_BLOCKS)
 expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const ExpandArgs& p = P.a;
@@ -99,27 +110,7 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
   const int ntl = min(P.tiles_total, t_begin + P.tiles_per_cta) - t_begin;
 #define LORA_TILE(t) (t_begin + (t))
 #endif
-
   if (ntl <= 0) return;
-  // Rows of a block slot start at slot*128: fetch their sorted rows and tokens
-  // while the tables are read.
-  const bool block_slot = slot < (p.tok + kExBM - 1) / kExBM;
-  int spec_srow = 0, spec_tok = 0;
-  if (tid < kExBM && block_slot) {
-    spec_srow = min(slot * kExBM + tid, p.tok - 1);
-    if (P.row_list) spec_srow = clampi(__ldg(P.row_list + spec_srow), 0, p.tok - 1);
-    spec_tok = p.permutation ? clampi(__ldg(p.permutation + spec_srow), 0, p.tok - 1)
-                             : spec_srow;
-  }
-  PieceInfo pc;
-  const int32_t* indptr = P.vseg_indptr ? P.vseg_indptr : p.seg_indptr;
-  if (!find_piece_warp(indptr, P.vseg_indptr ? nullptr : p.weight_indices, p.scalings,
-                       P.nvseg, p.L, p.tok, kExBM, slot, pc))
-    return;
-  const int rows = pc.hi - pc.lo;
-  const int adapter = pc.adapter;
-  const float scale = pc.per_adapter;
-  if (scale == 0.f) return;  // zero scaling: the rows stay bit-identical
 
   // ---- shared memory: [base ring][rank activations S x][B ring][row tables][barriers]
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -141,6 +132,57 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * P.b_stages + 5 +
                                                     2 * P.base_stages);
 
+  // barriers and TMEM first, so that their latency overlaps the table reads
+  if (tid == 0) {
+    for (int s = 0; s < P.b_stages; ++s) {
+      mbar_init(bfull0 + 8 * s, 1);
+      mbar_init(bempty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, kExConsumers);
+    }
+    mbar_init(rin_bar, kExProducers);
+    for (int s = 0; s < P.base_stages; ++s) {
+      mbar_init(xfull0 + 8 * s, kExProducers);
+      mbar_init(xempty0 + 8 * s, kExConsumers);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&P.tmap_B);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), kExTmemCols);
+    tmem_relinquish();
+  }
+
+  // Rows of a block slot start at slot*128: fetch their sorted rows and tokens
+  // while the tables are read.
+  const bool block_slot = slot < (p.tok + kExBM - 1) / kExBM;
+  int spec_srow = 0, spec_tok = 0;
+  if (tid < kExBM && block_slot) {
+    spec_srow = min(slot * kExBM + tid, p.tok - 1);
+    if (P.row_list) spec_srow = clampi(__ldg(P.row_list + spec_srow), 0, p.tok - 1);
+    spec_tok = p.permutation ? clampi(__ldg(p.permutation + spec_srow), 0, p.tok - 1)
+                             : spec_srow;
+  }
+  PieceInfo pc;
+  const int32_t* indptr = P.vseg_indptr ? P.vseg_indptr : p.seg_indptr;
+  const bool have = find_piece_warp(indptr, P.vseg_indptr ? nullptr : p.weight_indices,
+                                    p.scalings, P.nvseg, p.L, p.tok, kExBM, slot, pc);
+  // no rows here, or a zero scaling (the rows then stay bit-identical): leave
+  if (!have || pc.per_adapter == 0.f) {
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+      tc_fence_after();
+      tmem_dealloc(*tmem_slot, kExTmemCols);
+    }
+    return;
+  }
+  const int rows = pc.hi - pc.lo;
+  const int adapter = pc.adapter;
+  const float scale = pc.per_adapter;
+
   const int off0 = p.slices.off[0];
   const int64_t n_tot = p.slices.off[p.S] - off0;
 
@@ -155,27 +197,6 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
       srow_of[m] = sr;
       trow[m] = p.permutation ? clampi(__ldg(p.permutation + sr), 0, p.tok - 1) : sr;
     }
-  }
-  if (tid == 0) {
-    for (int s = 0; s < P.b_stages; ++s) {
-      mbar_init(bfull0 + 8 * s, 1);
-      mbar_init(bempty0 + 8 * s, 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(tfull0 + 8 * b, 1);
-      mbar_init(tempty0 + 8 * b, kExBM);
-    }
-    mbar_init(rin_bar, kExBM);
-    for (int s = 0; s < P.base_stages; ++s) {
-      mbar_init(xfull0 + 8 * s, kExBM);
-      mbar_init(xempty0 + 8 * s, kExBM);
-    }
-    fence_mbar_init();
-    tma_prefetch_desc(&P.tmap_B);
-  }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), kExTmemCols);
-    tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
@@ -237,10 +258,12 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
       }
     }
     __syncwarp();
-  } else if (warp >= 5) {
+  } else if (warp >= 9) {
     // =========================== producers (128 threads)
-    const int pt = tid - 5 * 32;
-    // (1) rank activations of every slice, zero-filled beyond r (thread = row)
+    const int pt = tid - 9 * 32;
+    // (1) rank activations of every slice, zero-filled beyond r (thread = row);
+    //     committed as their own cp.async group and waited for only after the
+    //     first base tiles are on their way
     {
       const int m = pt;
       const bool row_ok = m < rows;
@@ -257,11 +280,9 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
         }
       }
       cp_async_commit();
-      cp_async_wait<0>();
-      fence_proxy_async_smem();  // read by the MMA through the async proxy
-      mbar_arrive(rin_bar);
     }
     // (2) base tiles: chunk u = j*128 + pt -> row u / kExCh, logical chunk u % kExCh
+    const int pre = min(P.base_stages, ntl);
     for (int t = 0; t < ntl && ok; ++t) {
       const int s = t % P.base_stages;
       if (t >= P.base_stages) ok = mbar_wait(xempty0 + 8 * s, ((t / P.base_stages) - 1) & 1);
@@ -284,13 +305,21 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
                     in ? 16u : 0u);
       }
       cp_async_arrive_noinc(xfull0 + 8 * s);
+      cp_async_commit();
+      if (t == pre - 1) {
+        // the rank-activation group is older than the `pre` tile groups
+        cp_async_wait_dyn(pre);
+        fence_proxy_async_smem();  // read by the MMA through the async proxy
+        mbar_arrive(rin_bar);
+      }
     }
     cp_async_wait<0>();
   } else {
-    // =========================== consumers (warps 1-4)
+    // =========================== consumers (warps 1-8)
     const int quarter = warp & 3;
+    const int half = (warp - 1) >> 2;
     const int m = quarter * 32 + lane;  // accumulator row of this thread
-    const int ct = tid - 32;            // 0..127 for the coalesced phase
+    const int ct = tid - 32;            // 0..255 for the coalesced phase
     for (int t = 0; t < ntl; ++t) {
       const int s = t % P.base_stages, buf = t & 1;
       if (ok) ok = mbar_wait(xfull0 + 8 * s, (t / P.base_stages) & 1);
@@ -301,49 +330,64 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
       tile_info(t, q, c0);
       uint8_t* stage_p = smem + (base_ring - sbase) + s * kExStageBytes;
       const uint32_t tacc = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * kExBN;
-      // (a) row-per-thread: base + scaling * acc, in place in shared memory
-#pragma unroll 1
-      for (int cc = 0; cc < kExBN / 16; ++cc) {
-        float v[16];
+      // (a) row-per-thread on this warp's half of the columns: base + scaling * acc.
+      //     TMEM loads go out kExLdBatch chunks at a time, one wait per batch.
+      constexpr int kHalfChunks = kExBN / 32;  // 16-column TMEM chunks per half
+#pragma unroll
+      for (int k0 = 0; k0 < kHalfChunks; k0 += kExLdBatch) {
+        float v[kExLdBatch][16];
         if (ok) {
-          tmem_ld16(tacc + cc * 16, v);
+#pragma unroll
+          for (int k = 0; k < kExLdBatch; ++k)
+            tmem_ld16(tacc + (half * kHalfChunks + k0 + k) * 16, v[k]);
           tmem_ld_wait();
         }
         if (ok && m < rows) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int c = 2 * cc + h;
-            uint4* ptr = reinterpret_cast<uint4*>(stage_p + m * (kExBN * 2) +
-                                                  ((c ^ (m & (kExCh - 1))) << 4));
-            uint4 w = *ptr;
-            uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
+          for (int k = 0; k < kExLdBatch; ++k) {
+            const int cc = half * kHalfChunks + k0 + k;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 b = E::u32_to_f2(wv[e]);
-              wv[e] = E::f2_to_u32(fmaf(scale, v[8 * h + 2 * e], b.x),
-                                   fmaf(scale, v[8 * h + 2 * e + 1], b.y));
+            for (int h = 0; h < 2; ++h) {
+              const int c = 2 * cc + h;
+              uint4* ptr = reinterpret_cast<uint4*>(stage_p + m * (kExBN * 2) +
+                                                    ((c ^ (m & (kExCh - 1))) << 4));
+              uint4 w = *ptr;
+              uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 b = E::u32_to_f2(wv[e]);
+                wv[e] = E::f2_to_u32(fmaf(scale, v[k][8 * h + 2 * e], b.x),
+                                     fmaf(scale, v[k][8 * h + 2 * e + 1], b.y));
+              }
+              *ptr = w;
             }
-            *ptr = w;
           }
         }
       }
       tc_fence_before();
       mbar_arrive(tempty0 + 8 * buf);
-      named_bar_sync(1, kExBM);  // every row of the tile is updated
-      // (b) coalesced write-back: chunk u = j*128 + ct -> row u / kExCh, chunk u % kExCh
+      named_bar_sync(1, kExConsumers);  // every row of the tile is updated
+      // (b) coalesced write-back: chunk u = j*256 + ct -> row u / kExCh, chunk u % kExCh;
+      //     all shared-memory reads first, then the stores
       const int cend = p.slices.off[q + 1];
       if (ok) {
-#pragma unroll 4
-        for (int j = 0; j < kExCh; ++j) {
-          const int u = j * kExBM + ct;
+        constexpr int kPer = (kExBM * kExCh) / kExConsumers;
+        uint4 w[kPer];
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+          const int u = j * kExConsumers + ct;
+          const int row = u / kExCh, c = u % kExCh;
+          w[j] = *reinterpret_cast<const uint4*>(stage_p + row * (kExBN * 2) +
+                                                 ((c ^ (row & (kExCh - 1))) << 4));
+        }
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+          const int u = j * kExConsumers + ct;
           const int row = u / kExCh, c = u % kExCh;
           const int col = c0 + 8 * c;
-          if (row < rows && col < cend) {
-            const uint4 w = *reinterpret_cast<const uint4*>(stage_p + row * (kExBN * 2) +
-                                                            ((c ^ (row & (kExCh - 1))) << 4));
+          if (row < rows && col < cend)
             *reinterpret_cast<uint4*>(p.base + static_cast<int64_t>(trow[row]) * p.ld_base +
-                                      col) = w;
-          }
+                                      col) = w[j];
         }
       }
       mbar_arrive(xempty0 + 8 * s);  // the stage's shared memory may be refilled

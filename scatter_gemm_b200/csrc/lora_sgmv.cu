@@ -236,7 +236,7 @@ lora_status shrink_tc(const lora::ShrinkArgs& a, lora_dtype dt, const Grouping& 
   // widest stage (64-K sub-tiles of x and A) that still leaves two stages, and
   // room for the split-K partial, inside the shared-memory budget
   const int budget = (LORA_SHRINK_CTAS_PER_SM >= 2 && P.npad <= 128 ? 110 : 220) * 1024;
-  const size_t part_bytes = sizeof(float) * lora::kTcBM * (P.npad + 1);
+  const size_t part_bytes = sizeof(float) * lora::kTcBM * (P.npad + 4);
   int nsub = lora::kTcMaxNSub;
   for (;; nsub /= 2) {
     const int sb = nsub * (lora::kTcBM * 128 + P.npad * 128);
@@ -252,6 +252,10 @@ lora_status shrink_tc(const lora::ShrinkArgs& a, lora_dtype dt, const Grouping& 
   // (expected pieces: one per 128 rows plus about half a piece per segment),
   // keeping at least four stages of K per CTA.  (Splitting further, to fill
   // every resident CTA slot, measured slower: more partials to reduce.)
+  if (!encode_2d(&P.tmap_A, dt, a.A, a.K, static_cast<uint64_t>(a.L) * a.S * a.rs,
+                 static_cast<uint64_t>(a.K) * 2, lora::kTcAtomK, P.npad,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return LORA_ERR_CUDA;
   const size_t smem_need = static_cast<size_t>(P.stages) * P.stage_bytes + 1024 +
                            8 * (2 * P.stages + 2) + 8 * lora::kTcBM + 16;
   const int est = (a.tok + lora::kTcBM - 1) / lora::kTcBM + (P.vseg_indptr ? a.L : a.nseg) / 2;
@@ -262,10 +266,6 @@ lora_status shrink_tc(const lora::ShrinkArgs& a, lora_dtype dt, const Grouping& 
   P.csplit = cs;
   P.kb_per = (P.nkb + cs - 1) / cs;
   P.idesc = lora::make_idesc_f16(dt == LORA_BF16 ? 1 : 0, lora::kTcBM, P.npad);
-  if (!encode_2d(&P.tmap_A, dt, a.A, a.K, static_cast<uint64_t>(a.L) * a.S * a.rs,
-                 static_cast<uint64_t>(a.K) * 2, lora::kTcAtomK, P.npad,
-                 CU_TENSOR_MAP_SWIZZLE_128B))
-    return LORA_ERR_CUDA;
 
   const size_t smem = smem_need;
   const long slots = lora::num_piece_slots(a.tok, P.nvseg, lora::kTcBM);
@@ -360,7 +360,7 @@ lora_status expand_tc(const lora::ExpandArgs& a, lora_dtype dt, const Grouping& 
   const int ctas_per_sm = (LORA_EXPAND_CTAS_PER_SM >= 2 && lora::kExTmemCols <= 256) ? 2 : 1;
   const size_t cap = (ctas_per_sm >= 2 ? 113 : 225) * 1024;
   P.base_stages = 2;
-  while (P.base_stages < 8 && total(P.base_stages + 1) <= cap) ++P.base_stages;
+  while (P.base_stages < 7 && total(P.base_stages + 1) <= cap) ++P.base_stages;
   if (total(P.base_stages) > 225 * 1024) return LORA_ERR_UNSUPPORTED;
   size_t smem = total(P.base_stages);
   // keep the CTAs per SM within TMEM: 512 columns / kExTmemCols

@@ -76,6 +76,33 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
   const int split = blockIdx.x % P.csplit;
   const int slot = blockIdx.x / P.csplit;
 
+  // ---- shared memory carve-up (1024-aligned stages, then barriers)
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t x_bytes = kTcNSub * kTcBM * 128;  // kTcNSub sub-tiles of 128 rows x 128 B
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.stages * P.stage_bytes);
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = full0 + 8 * P.stages;
+  const uint32_t done_bar = empty0 + 8 * P.stages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * P.stages + 1);
+  int64_t* xrow_tok = reinterpret_cast<int64_t*>(bars + 2 * P.stages + 2);  // [128] x row index
+
+  // barriers and TMEM first, so that their latency overlaps the table reads
+  if (tid == 0) {
+    for (int s = 0; s < P.stages; ++s) {
+      mbar_init(full0 + 8 * s, kTcBM + 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(done_bar, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&P.tmap_A);
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(tmem_slot), P.tmem_cols);
+    tmem_relinquish();
+  }
+
   // ---- piece of this cluster (identical in all its CTAs).  Rows of a block
   // slot start at slot*128, so their tokens are fetched while the tables are read.
   const bool block_slot = slot < (p.tok + kTcBM - 1) / kTcBM;
@@ -88,22 +115,18 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
   PieceInfo pc;
   const int32_t* indptr = P.vseg_indptr ? P.vseg_indptr : p.seg_indptr;
   if (!find_piece_warp(indptr, P.vseg_indptr ? nullptr : p.weight_indices, nullptr, P.nvseg,
-                       p.L, p.tok, kTcBM, slot, pc))
+                       p.L, p.tok, kTcBM, slot, pc)) {
+    // no rows here (the same answer in every CTA of the cluster): give TMEM back
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 4) {
+      tc_fence_after();
+      tmem_dealloc(*tmem_slot, P.tmem_cols);
+    }
     return;
+  }
   const int rows = pc.hi - pc.lo;
   const int adapter = pc.adapter;
-
-  // ---- shared memory carve-up (1024-aligned stages, then barriers)
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  const uint32_t sbase = smem_u32(smem);
-  const uint32_t x_bytes = kTcNSub * kTcBM * 128;  // kTcNSub sub-tiles of 128 rows x 128 B
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.stages * P.stage_bytes);
-  const uint32_t full0 = smem_u32(bars);
-  const uint32_t empty0 = full0 + 8 * P.stages;
-  const uint32_t done_bar = empty0 + 8 * P.stages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * P.stages + 1);
-  int64_t* xrow_tok = reinterpret_cast<int64_t*>(bars + 2 * P.stages + 2);  // [128] x row index
 
   // K blocks of this CTA.  Interleaved over the cluster (CTA c takes blocks
   // c, c+C, c+2C, ...), so the C co-scheduled CTAs of a piece read C adjacent
@@ -128,19 +151,6 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
       xrow_tok[m] = p.permutation ? clampi(__ldg(p.permutation + srow), 0, p.tok - 1) : srow;
     }
   }
-  if (tid == 0) {
-    for (int s = 0; s < P.stages; ++s) {
-      mbar_init(full0 + 8 * s, kTcBM + 1);
-      mbar_init(empty0 + 8 * s, 1);
-    }
-    mbar_init(done_bar, 1);
-    fence_mbar_init();
-    tma_prefetch_desc(&P.tmap_A);
-  }
-  if (warp == 4) {
-    tmem_alloc(smem_u32(tmem_slot), P.tmem_cols);
-    tmem_relinquish();
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -148,11 +158,24 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
   bool ok = true;
 
   if (warp < 4) {
-    // =========================== producer: gather x rows, TMA the A block
-    // chunk u = j*128 + tid of a stage -> row u/8, 16-byte chunk u%8: every warp
-    // instruction reads 4 rows x 128 contiguous bytes
+    // =========================== producer: gather x rows and the A block
+    // A stage holds NSUB sub-tiles of 16-byte chunks; chunk u = j*128 + tid ->
+    // row u / (8*NSUB), chunk u % (8*NSUB).  The chunk column of a thread is the
+    // same for every row and stage, and its x rows are the same for every stage,
+    // so their addresses are formed once.  Thread 0 also loads the stage's A
+    // block with TMA (measured faster than gathering A with cp.async).
+    constexpr int CPR = 8 * kTcNSub;              // 16-byte chunks per row per stage
+    constexpr int RSTEP = kTcBM / CPR;            // rows between a thread's chunks
+    const int cc = tid % CPR;                     // this thread's chunk column
+    const int rr = tid / CPR;                     // ... and first row
+    const uint32_t sub_off = (cc >> 3) * (kTcBM * 128);  // x sub-tile of this chunk
     const uint32_t a_sub = P.npad * 128;  // one 64-K sub-tile of A
     const uint32_t a_bytes = kTcNSub * a_sub;
+    // gathered x row of each of this thread's CPR rows (rows past the piece are
+    // never read)
+    const uint16_t* xr[CPR];
+#pragma unroll
+    for (int j = 0; j < CPR; ++j) xr[j] = p.x + xrow_tok[rr + j * RSTEP] * p.ld_x;
     const int lag = P.stages - 1;
     for (int i = 0; i < nk && ok; ++i) {
       const int s = i % P.stages;
@@ -167,18 +190,14 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
           tma_load_2d(xs + x_bytes + sub * a_sub, &P.tmap_A, full0 + 8 * s, k0 + sub * kTcAtomK,
                       adapter * p.S * p.rs);
       }
-      // chunk u = j*128 + tid -> row u / (BK/8), 16-byte chunk u % (BK/8): a warp
-      // instruction reads 512 / (BK/8 * 16 / 512) rows of contiguous bytes
-#pragma unroll 8
-      for (int j = 0; j < kTcBK / 8; ++j) {
-        const int u = j * kTcBM + tid;
-        const int row = u / (kTcBK / 8), c = u % (kTcBK / 8);
-        const int k = k0 + 8 * c;
-        const bool in = row < rows && k < p.K;
-        const uint32_t dst = xs + (c >> 3) * (kTcBM * 128) + row * 128 +
-                             (((c & 7) ^ (row & 7)) << 4);
-        cp_async_16(dst, in ? static_cast<const void*>(p.x + xrow_tok[row] * p.ld_x + k)
-                            : static_cast<const void*>(p.x),
+      const int k = k0 + 8 * cc;
+      const bool k_in = k < p.K;
+#pragma unroll
+      for (int j = 0; j < CPR; ++j) {
+        const int row = rr + j * RSTEP;
+        const bool in = k_in && row < rows;
+        const uint32_t dst = xs + sub_off + row * 128 + (((cc & 7) ^ (row & 7)) << 4);
+        cp_async_16(dst, in ? static_cast<const void*>(xr[j] + k) : static_cast<const void*>(p.x),
                     in ? 16u : 0u);
       }
       cp_async_commit();
@@ -220,8 +239,11 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
   }
 
   // =========================== epilogue (warps 0-3: one accumulator row per thread)
-  float* part = reinterpret_cast<float*>(smem);  // split-K partial, reuses the stage ring
-  const int pstride = P.npad + 1;
+  // Split-K partials reuse the stage ring as [128][npad + 4] fp32: 16-byte rows
+  // whose stride (4 or 20 words mod 32) keeps the row-per-thread 16-byte
+  // stores free of bank conflicts.
+  float* part = reinterpret_cast<float*>(smem);
+  const int pstride = P.npad + 4;
   if (warp < 4) {
     if (ok) ok = mbar_wait(done_bar, 0);
     ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
@@ -250,8 +272,10 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
           }
         }
       } else {
+        float4* dst = reinterpret_cast<float4*>(part + m * pstride + c0);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) part[m * pstride + c0 + i] = v[i];
+        for (int i = 0; i < 4; ++i)
+          dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
       }
     }
     tc_fence_before();
@@ -259,21 +283,42 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
 
   if (P.csplit > 1) {
     cluster_sync();  // every partial of the cluster is in shared memory
+    // CTA `split` owns rows [split*R, (split+1)*R); a thread sums one 4-column
+    // group over all C partials: the C remote 16-byte loads are issued back to
+    // back and only then added, in rank order (deterministic).
     const int R = kTcBM / P.csplit;
     const int r0 = split * R;
-    const int nv = p.S * p.r;
+    const int ng = P.npad / 4;
+    const int nvalid = p.S * p.rs;
     const uint32_t pbase = smem_u32(part);
-    for (int e = tid; e < R * nv; e += kTcThreads) {
-      const int row = r0 + e / nv;
-      const int v = e % nv;
-      const int n = (v / p.r) * p.rs + (v % p.r);
+    for (int e = tid; e < R * ng; e += kTcThreads) {
+      const int row = r0 + e / ng;
+      const int g = e % ng;
       if (row >= rows) continue;
-      const uint32_t off = pbase + 4u * static_cast<uint32_t>(row * pstride + n);
-      float sum = 0.f;
-      for (int q = 0; q < P.csplit; ++q) sum += ld_dsmem_f32(mapa_shared(off, q));
+      const uint32_t off = pbase + 4u * static_cast<uint32_t>(row * pstride + 4 * g);
+      float4 pv[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (q < P.csplit) pv[q] = ld_dsmem_v4(mapa_shared(off, q));
+      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        if (q < P.csplit) {
+          sum.x += pv[q].x;
+          sum.y += pv[q].y;
+          sum.z += pv[q].z;
+          sum.w += pv[q].w;
+        }
+      }
       const int orow_i = P.row_list ? clampi(__ldg(P.row_list + pc.lo + row), 0, p.tok - 1)
                                     : pc.lo + row;
-      if (ok) p.out[static_cast<int64_t>(orow_i) * p.ld_out + n] = E::f32_to_bits(sum);
+      uint16_t* orow = p.out + static_cast<int64_t>(orow_i) * p.ld_out;
+      const float sv[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int n = 4 * g + k;
+        if (ok && n < nvalid && (n % p.rs) < p.r) orow[n] = E::f32_to_bits(sv[k]);
+      }
     }
     cluster_sync();  // peers are done reading this CTA's partial
   }
