@@ -41,7 +41,7 @@
 namespace lora {
 
 #ifndef LORA_EXPAND_BN
-#define LORA_EXPAND_BN 128  // columns per tile (128 or 256)
+#define LORA_EXPAND_BN 128  // columns per tile (64, 128 or 256)
 #endif
 #ifndef LORA_EXPAND_LD_BATCH
 #define LORA_EXPAND_LD_BATCH 2  // 16-column TMEM loads in flight per consumer thread
@@ -59,7 +59,7 @@ constexpr int kExThreads = 32 + kExConsumers + kExProducers;
 constexpr int kExStageBytes = kExBM * kExBN * 2;  // one staged base tile
 constexpr int kExLdBatch = LORA_EXPAND_LD_BATCH;   // TMEM chunks loaded per wait
 static_assert((kExBN / 32) % kExLdBatch == 0, "batch must divide a half tile");
-static_assert(kExBN == 128 || kExBN == 256, "expand tile width");
+static_assert(kExBN == 64 || kExBN == 128 || kExBN == 256, "expand tile width");
 
 struct ExpandTcParams {
   CUtensorMap tmap_B;  // 2-D [L*N_tot rows, r cols] (row stride rs), box {rpad, 128}
@@ -112,7 +112,7 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
 #endif
   if (ntl <= 0) return;
 
-  // ---- shared memory: [base ring][rank activations S x][B ring][row tables][barriers]
+  // ---- shared memory: [base ring][rank activations S x][B ring][token of each row][barriers]
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -120,8 +120,7 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
   const uint32_t rin = base_ring + P.base_stages * kExStageBytes;
   const uint32_t bring = rin + p.S * P.rin_bytes;
   int* trow = reinterpret_cast<int*>(smem + (bring - sbase) + P.b_stages * P.btile_bytes);
-  int* srow_of = trow + kExBM;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(srow_of + kExBM);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(trow + kExBM);
   const uint32_t bfull0 = smem_u32(bars);
   const uint32_t bempty0 = bfull0 + 8 * P.b_stages;
   const uint32_t tfull0 = bempty0 + 8 * P.b_stages;  // 2 accumulator buffers
@@ -132,8 +131,9 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * P.b_stages + 5 +
                                                     2 * P.base_stages);
 
-  // barriers and TMEM first, so that their latency overlaps the table reads
-  if (tid == 0) {
+  // Barriers (one consumer thread) and TMEM (warp 0) first, in different warps,
+  // so that both overlap the table reads.
+  if (tid == 32) {
     for (int s = 0; s < P.b_stages; ++s) {
       mbar_init(bfull0 + 8 * s, 1);
       mbar_init(bempty0 + 8 * s, 1);
@@ -148,19 +148,21 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
       mbar_init(xempty0 + 8 * s, kExConsumers);
     }
     fence_mbar_init();
-    tma_prefetch_desc(&P.tmap_B);
   }
   if (warp == 0) {
+    if (lane == 0) tma_prefetch_desc(&P.tmap_B);
     tmem_alloc(smem_u32(tmem_slot), kExTmemCols);
     tmem_relinquish();
   }
 
-  // Rows of a block slot start at slot*128: fetch their sorted rows and tokens
-  // while the tables are read.
+  // Producer thread pt owns row pt of the piece.  Rows of a block slot start
+  // at slot*128: their sorted rows and tokens are fetched while the tables are read.
+  const bool producer = warp >= 9;
+  const int pt = tid - 9 * 32;
   const bool block_slot = slot < (p.tok + kExBM - 1) / kExBM;
   int spec_srow = 0, spec_tok = 0;
-  if (tid < kExBM && block_slot) {
-    spec_srow = min(slot * kExBM + tid, p.tok - 1);
+  if (producer && block_slot) {
+    spec_srow = min(slot * kExBM + pt, p.tok - 1);
     if (P.row_list) spec_srow = clampi(__ldg(P.row_list + spec_srow), 0, p.tok - 1);
     spec_tok = p.permutation ? clampi(__ldg(p.permutation + spec_srow), 0, p.tok - 1)
                              : spec_srow;
@@ -186,24 +188,6 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
   const int off0 = p.slices.off[0];
   const int64_t n_tot = p.slices.off[p.S] - off0;
 
-  if (tid < kExBM) {
-    const int m = tid;
-    if (block_slot) {
-      srow_of[m] = spec_srow;
-      trow[m] = spec_tok;
-    } else {
-      int sr = pc.lo + (m < rows ? m : 0);
-      if (P.row_list) sr = clampi(__ldg(P.row_list + sr), 0, p.tok - 1);
-      srow_of[m] = sr;
-      trow[m] = p.permutation ? clampi(__ldg(p.permutation + sr), 0, p.tok - 1) : sr;
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  bool ok = true;
-
   // tile t of this CTA -> (slice, first column)
   auto tile_info = [&](int t, int& q, int& c0) {
     const int g = LORA_TILE(t);
@@ -213,6 +197,68 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
       if (k < p.S && g >= P.tile_prefix[k]) q = k;
     c0 = p.slices.off[q] + (g - P.tile_prefix[q]) * kExBN;
   };
+  // base tile t into ring stage s: chunk u = j*128 + pt -> row u / kExCh,
+  // logical chunk u % kExCh (two 256-byte rows per warp instruction)
+  auto issue_tile = [&](int t, int s) {
+    int q, c0;
+    tile_info(t, q, c0);
+    const int cend = p.slices.off[q + 1];
+    const uint32_t stage = base_ring + s * kExStageBytes;
+#pragma unroll 4
+    for (int j = 0; j < kExCh; ++j) {
+      const int u = j * kExBM + pt;
+      const int row = u / kExCh, c = u % kExCh;
+      const int col = c0 + 8 * c;
+      const bool in = row < rows && col < cend;
+      cp_async_16(stage + row * (kExBN * 2) + ((c ^ (row & (kExCh - 1))) << 4),
+                  in ? static_cast<const void*>(p.base +
+                                                static_cast<int64_t>(trow[row]) * p.ld_base + col)
+                     : static_cast<const void*>(p.base),
+                  in ? 16u : 0u);
+    }
+  };
+  const int pre = min(P.base_stages, ntl);  // tiles issued before the CTA barrier
+
+  if (producer) {
+    // Row tables, then every load that needs no barrier goes out before the
+    // CTA-wide barrier: the rank activations of row pt (zero-filled beyond r,
+    // their own cp.async group) and the first `pre` base tiles (one group each).
+    const int m = pt;
+    int sr, tk;
+    if (block_slot) {
+      sr = spec_srow;
+      tk = spec_tok;
+    } else {
+      sr = pc.lo + (m < rows ? m : 0);
+      if (P.row_list) sr = clampi(__ldg(P.row_list + sr), 0, p.tok - 1);
+      tk = p.permutation ? clampi(__ldg(p.permutation + sr), 0, p.tok - 1) : sr;
+    }
+    trow[m] = tk;
+    const bool row_ok = m < rows;
+    const uint16_t* src0 = p.in_r + static_cast<int64_t>(sr) * p.ld_in;
+    const int nchunk = P.rpad / 8;
+    for (int q = 0; q < p.S; ++q) {
+      for (int c = 0; c < nchunk; ++c) {
+        const int left = p.r - 8 * c;
+        const uint32_t nb = row_ok ? static_cast<uint32_t>(max(0, min(left, 8)) * 2) : 0u;
+        const uint32_t dst = rin + q * P.rin_bytes + m * (P.rpad * 2) +
+                             (swz_chunk(c, m, P.rpad) << 4);
+        cp_async_16(dst, nb ? static_cast<const void*>(src0 + q * p.rs + 8 * c)
+                            : static_cast<const void*>(p.in_r), nb);
+      }
+    }
+    cp_async_commit();
+    named_bar_sync(2, kExProducers);  // trow of every row is in shared memory
+    for (int t = 0; t < pre; ++t) {
+      issue_tile(t, t);
+      cp_async_commit();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
 
   if (warp == 0) {
     // =========================== B tiles (TMA) and MMA issue
@@ -260,58 +306,24 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
     __syncwarp();
   } else if (warp >= 9) {
     // =========================== producers (128 threads)
-    const int pt = tid - 9 * 32;
-    // (1) rank activations of every slice, zero-filled beyond r (thread = row);
-    //     committed as their own cp.async group and waited for only after the
-    //     first base tiles are on their way
-    {
-      const int m = pt;
-      const bool row_ok = m < rows;
-      const uint16_t* src0 = p.in_r + static_cast<int64_t>(srow_of[m]) * p.ld_in;
-      const int nchunk = P.rpad / 8;
-      for (int q = 0; q < p.S; ++q) {
-        for (int c = 0; c < nchunk; ++c) {
-          const int left = p.r - 8 * c;
-          const uint32_t nb = row_ok ? static_cast<uint32_t>(max(0, min(left, 8)) * 2) : 0u;
-          const uint32_t dst = rin + q * P.rin_bytes + m * (P.rpad * 2) +
-                               (swz_chunk(c, m, P.rpad) << 4);
-          cp_async_16(dst, nb ? static_cast<const void*>(src0 + q * p.rs + 8 * c)
-                              : static_cast<const void*>(p.in_r), nb);
-        }
-      }
-      cp_async_commit();
+    // Publish what went out before the barrier, oldest group first: the rank
+    // activations (read by the MMA through the async proxy), then each early tile.
+    cp_async_wait_dyn(pre);
+    fence_proxy_async_smem();
+    mbar_arrive(rin_bar);
+    for (int t = 0; t < pre; ++t) {
+      cp_async_wait_dyn(pre - 1 - t);
+      mbar_arrive(xfull0 + 8 * t);
     }
-    // (2) base tiles: chunk u = j*128 + pt -> row u / kExCh, logical chunk u % kExCh
-    const int pre = min(P.base_stages, ntl);
-    for (int t = 0; t < ntl && ok; ++t) {
+    // The remaining tiles: completion reaches the consumers through
+    // cp.async.mbarrier.arrive, so the producers never block on a tile.
+    for (int t = pre; t < ntl && ok; ++t) {
       const int s = t % P.base_stages;
-      if (t >= P.base_stages) ok = mbar_wait(xempty0 + 8 * s, ((t / P.base_stages) - 1) & 1);
+      ok = mbar_wait(xempty0 + 8 * s, ((t / P.base_stages) - 1) & 1);
       if (!ok) break;
-      int q, c0;
-      tile_info(t, q, c0);
-      const int cend = p.slices.off[q + 1];
-      const uint32_t stage = base_ring + s * kExStageBytes;
-#pragma unroll 4
-      for (int j = 0; j < kExCh; ++j) {
-        const int u = j * kExBM + pt;
-        const int row = u / kExCh, c = u % kExCh;
-        const int col = c0 + 8 * c;
-        const bool in = row < rows && col < cend;
-        cp_async_16(stage + row * (kExBN * 2) + ((c ^ (row & (kExCh - 1))) << 4),
-                    in ? static_cast<const void*>(p.base +
-                                                  static_cast<int64_t>(trow[row]) * p.ld_base +
-                                                  col)
-                       : static_cast<const void*>(p.base),
-                    in ? 16u : 0u);
-      }
+      issue_tile(t, s);
       cp_async_arrive_noinc(xfull0 + 8 * s);
       cp_async_commit();
-      if (t == pre - 1) {
-        // the rank-activation group is older than the `pre` tile groups
-        cp_async_wait_dyn(pre);
-        fence_proxy_async_smem();  // read by the MMA through the async proxy
-        mbar_arrive(rin_bar);
-      }
     }
     cp_async_wait<0>();
   } else {

@@ -351,7 +351,7 @@ lora_status expand_tc(const lora::ExpandArgs& a, lora_dtype dt, const Grouping& 
   // shared memory: base ring, rank activations, B ring, row tables, barriers
   P.b_stages = LORA_EXPAND_B_STAGES;
   const size_t fixed = static_cast<size_t>(a.S) * P.rin_bytes +
-                       static_cast<size_t>(P.b_stages) * P.btile_bytes + 1024 + 1024 + 16;
+                       static_cast<size_t>(P.b_stages) * P.btile_bytes + 1024 + 512 + 16;
   auto total = [&](int bs) {
     return ((static_cast<size_t>(bs) * lora::kExStageBytes + 1023) & ~size_t(1023)) + fixed +
            8 * (2 * P.b_stages + 5 + 2 * bs);

@@ -88,21 +88,30 @@ struct PieceInfo {
 constexpr int kTabPerLane = 8;
 constexpr int kTabMax = 32 * kTabPerLane;
 
+// Value of table entry i, held as v[i / 32] by lane i % 32 (i uniform over the
+// warp).  Every register is shuffled with a constant index and the result is
+// picked by a select chain: indexing v with i / 32 would put the table in
+// local memory, which misses L1 when shared memory fills the SM.
 __device__ __forceinline__ int pick(const int (&v)[kTabPerLane], int i) {
-  // value of table entry i held as v[i / 32] by lane i % 32 (i uniform over the warp)
+  const int src = i & 31, k = i >> 5;
   int r = 0;
 #pragma unroll
-  for (int k = 0; k < kTabPerLane; ++k)
-    if ((i >> 5) == k) r = v[k];
-  return __shfl_sync(0xffffffffu, r, i & 31);
+  for (int j = 0; j < kTabPerLane; ++j) {
+    const int t = __shfl_sync(0xffffffffu, v[j], src);
+    r = (k == j) ? t : r;
+  }
+  return r;
 }
 
 __device__ __forceinline__ float pickf(const float (&v)[kTabPerLane], int i) {
+  const int src = i & 31, k = i >> 5;
   float r = 0.f;
 #pragma unroll
-  for (int k = 0; k < kTabPerLane; ++k)
-    if ((i >> 5) == k) r = v[k];
-  return __shfl_sync(0xffffffffu, r, i & 31);
+  for (int j = 0; j < kTabPerLane; ++j) {
+    const float t = __shfl_sync(0xffffffffu, v[j], src);
+    r = (k == j) ? t : r;
+  }
+  return r;
 }
 
 __device__ __forceinline__ bool find_piece_warp(const int32_t* __restrict__ seg_indptr,
