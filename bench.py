@@ -306,14 +306,19 @@ def run_ours(args, rank, world, device):
     if rank != 0:
         return
     peak, peak_kind = measured_peaks()
-    med = np.median(t, axis=0)  # per call, ms
+    # per call, ms: means (CUDA event timestamps tick in ~2 us steps, so medians
+    # of single calls are quantized; the mean over steps is not)
+    med = np.median(t, axis=0)
+    avg = t.mean(axis=0)
     detail = []
     fr = []
     for j, dp in enumerate(probs):
-        s_ms, e_ms = med[2 * j], med[2 * j + 1]
+        s_ms, e_ms = avg[2 * j], avg[2 * j + 1]
         gbs = (dp.bytes_shrink + dp.bytes_expand) / ((s_ms + e_ms) * 1e-3) / 1e9
         detail.append({"tok": dp.p.tok,
                        "shrink_us": round(s_ms * 1e3, 2), "expand_us": round(e_ms * 1e3, 2),
+                       "shrink_us_median": round(med[2 * j] * 1e3, 2),
+                       "expand_us_median": round(med[2 * j + 1] * 1e3, 2),
                        "shrink_gbs": round(dp.bytes_shrink / (s_ms * 1e-3) / 1e9, 1),
                        "expand_gbs": round(dp.bytes_expand / (e_ms * 1e-3) / 1e9, 1),
                        "gbs": round(gbs, 1)})

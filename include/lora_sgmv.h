@@ -85,7 +85,8 @@ enum {
   LORA_PATH_GENERAL = 1, /* element-aligned CUDA-core kernel                       */
   LORA_PATH_TENSOR = 2,  /* tcgen05 tensor-core kernel (16-byte-aligned inputs)     */
   LORA_PATH_GROUPED = 4, /* rows grouped by adapter first (workspace, many segments) */
-  LORA_PATH_SPLITK = 8   /* shrink K range split over a thread-block cluster        */
+  LORA_PATH_SPLITK = 8,  /* shrink K range split over a thread-block cluster        */
+  LORA_PATH_FUSED = 16   /* lora_shrink_expand ran both ops in one launch            */
 };
 
 /* Limits of this build. */
@@ -250,6 +251,61 @@ LORA_API lora_status lora_shrink_static_scratch(const void* x, int64_t ld_x, con
                                                 int64_t ld_out, int tok, int K, int S, int r,
                                                 int rs, int nseg, int L, lora_dtype dtype,
                                                 void* stream);
+
+/* lora_shrink_expand -- the pair in one call: lora_shrink into out_r, then
+ * lora_expand with in_r = out_r (the rank activations rounded once to the
+ * element type in between, as in the sgl-kernel-xpu page, section "Summary").
+ *   x, A_stack, seg_indptr, weight_indices, permutation, out_r, ld_out: as lora_shrink
+ *   B_stack, slice_offsets (HOST), scalings, base_out, ld_base:          as lora_expand
+ * out_r [tok, ld_out >= S*rs] is written (valid columns j < r of the rows in
+ * segments) and base_out updated, with the results of the two calls made
+ * one after the other, up to the fp32 summation order of the shrink.  For
+ * decode-sized batches (tok <= 512, few segments, 16-byte-aligned tensors)
+ * one kernel does both: a thread-block cluster per piece runs a split-K
+ * shrink, shares the rounded rank activations through distributed shared
+ * memory and runs the expand of that piece (LORA_PATH_FUSED).  Otherwise the
+ * two calls run in sequence on the stream (using `workspace` as they do).
+ * Errors: those of lora_shrink and lora_expand. */
+LORA_API lora_status lora_shrink_expand(const void* x, int64_t ld_x, const void* A_stack,
+                                        const void* B_stack, const int32_t* seg_indptr,
+                                        const int32_t* weight_indices,
+                                        const int32_t* permutation,
+                                        const int32_t* slice_offsets, const float* scalings,
+                                        void* out_r, int64_t ld_out, void* base_out,
+                                        int64_t ld_base, int tok, int K, int S, int r, int rs,
+                                        int nseg, int L, lora_dtype dtype, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
+/* ---- 64-bit index tables ------------------------------------------------
+ * lora_shrink_i64 / lora_expand_i64 take seg_indptr, weight_indices and
+ * permutation as int64_t (the default index type of PyTorch), as the
+ * ring-attention page ("Tests") does for its cu_seqlens; everything else is
+ * exactly lora_shrink / lora_expand.  One small kernel narrows the three
+ * tables into the front of `workspace` (device memory, 16-byte aligned, owned
+ * by the caller, stream-ordered like the call), and the call then continues
+ * on the int32 path with the rest of the workspace.  Values outside int32
+ * saturate; like any other invalid table value they are clamped by the
+ * kernels and reported by lora_validate on the narrowed tables.
+ * workspace_bytes must be at least lora_index64_workspace_size(tok, nseg),
+ * else LORA_ERR_INVALID_ARGUMENT; adding lora_workspace_size(tok, nseg, L)
+ * keeps the adapter-grouped schedule.  The narrowing counts in
+ * lora_launch_count. */
+LORA_API size_t lora_index64_workspace_size(int tok, int nseg);
+
+LORA_API lora_status lora_shrink_i64(const void* x, int64_t ld_x, const void* A_stack,
+                                     const int64_t* seg_indptr, const int64_t* weight_indices,
+                                     const int64_t* permutation, void* out_r, int64_t ld_out,
+                                     int tok, int K, int S, int r, int rs, int nseg, int L,
+                                     lora_dtype dtype, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
+LORA_API lora_status lora_expand_i64(const void* in_r, int64_t ld_in, const void* B_stack,
+                                     const int64_t* seg_indptr, const int64_t* weight_indices,
+                                     const int64_t* permutation, const int32_t* slice_offsets,
+                                     const float* scalings, void* base_out, int64_t ld_base,
+                                     int tok, int S, int r, int rs, int nseg, int L,
+                                     lora_dtype dtype, void* workspace, size_t workspace_bytes,
+                                     void* stream);
 
 /* Kernel path (LORA_PATH_* bits) chosen by the last lora_shrink / lora_expand
  * call made on this host thread; 0 if none launched a kernel. */

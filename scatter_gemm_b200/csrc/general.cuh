@@ -184,6 +184,29 @@ expand_general_kernel(const ExpandArgs p) {
 // ---------------------------------------------------------------------------
 __global__ void set_word_kernel(int32_t* __restrict__ w, int32_t v) { *w = v; }
 
+// Narrows three int64 index tables to int32, saturating, one thread per
+// destination word.  Table a (na entries) goes to out[0..pa), table b (nb
+// entries) to out[pa..pa+pb), table c (nc entries) to out[pa+pb..pa+pb+nc);
+// pa >= na and pb >= nb are padded sizes whose extra words are set to 0.
+__global__ void narrow_index_kernel(const int64_t* __restrict__ a, int na, int pa,
+                                    const int64_t* __restrict__ b, int nb, int pb,
+                                    const int64_t* __restrict__ c, int nc,
+                                    int32_t* __restrict__ out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t n = static_cast<int64_t>(pa) + pb + nc;
+  if (i >= n) return;
+  int64_t v = 0;
+  if (i < pa) {
+    if (i < na) v = __ldg(a + i);
+  } else if (i < static_cast<int64_t>(pa) + pb) {
+    const int64_t j = i - pa;
+    if (j < nb) v = __ldg(b + j);
+  } else {
+    v = __ldg(c + (i - pa - pb));
+  }
+  out[i] = v > INT32_MAX ? INT32_MAX : (v < INT32_MIN ? INT32_MIN : static_cast<int32_t>(v));
+}
+
 __global__ void validate_kernel(const int32_t* __restrict__ seg_indptr,
                                 const int32_t* __restrict__ weight_indices,
                                 const int32_t* __restrict__ perm, int tok, int nseg, int L,

@@ -24,6 +24,7 @@
 #include "common.cuh"
 #include "embedding.cuh"
 #include "expand_tc.cuh"
+#include "fused_tc.cuh"
 #include "general.cuh"
 #include "group.cuh"
 #include "sched.cuh"
@@ -70,6 +71,9 @@ struct DeviceFacts {
   std::atomic<int> ready{0};
   int sms = 148;
   int max_cluster = 8;  // largest K-split cluster the shrink may use
+  // clusters of 1, 2, 4, 8, 16 CTAs of the fused kernel (one CTA per SM) that
+  // can be resident at once
+  int fused_clusters[5] = {0, 0, 0, 0, 0};
 };
 DeviceFacts g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -91,6 +95,10 @@ void set_kernel_attrs() {
                        227 * 1024);
   cudaFuncSetAttribute(lora::expand_general_kernel<E>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  cudaFuncSetAttribute(lora::fused_tc_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       227 * 1024);
+  cudaFuncSetAttribute(lora::fused_tc_kernel<E>, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                       1);
 }
 
 const DeviceFacts* device_facts() {
@@ -125,6 +133,17 @@ const DeviceFacts* device_facts() {
         nclusters > 0)
       f.max_cluster = 16;
     cudaGetLastError();  // the probe above must not leave a sticky launch error
+    for (int i = 0; i < 5; ++i) {
+      attr[0].val.clusterDim.x = 1u << i;
+      cfg.gridDim = dim3(16u << i);
+      cfg.blockDim = dim3(lora::kFuThreads);
+      cfg.dynamicSmemBytes = 200 * 1024;
+      int nc = 0;
+      if (cudaOccupancyMaxActiveClusters(&nc, lora::fused_tc_kernel<lora::Bf16>, &cfg) ==
+          cudaSuccess)
+        f.fused_clusters[i] = nc;
+      cudaGetLastError();
+    }
     f.ready.store(1, std::memory_order_release);
   }
   return &f;
@@ -178,6 +197,68 @@ inline size_t a16(size_t n) { return (n + 3) / 4 * 4; }  // ints -> multiple of 
 size_t workspace_ints(int tok, int nseg, int L) {
   return a16(static_cast<size_t>(L) + 1) + a16(static_cast<size_t>(nseg)) +
          a16(static_cast<size_t>(tok));
+}
+
+// Narrowed int64 tables at the front of an *_i64 call's workspace:
+// [seg_indptr (nseg+1)][weight_indices (nseg)][permutation (tok)], each padded
+// to 16 bytes, so the rest of the workspace stays 16-byte aligned.
+size_t index64_bytes(int tok, int nseg) {
+  return 4 * (a16(static_cast<size_t>(nseg) + 1) + a16(static_cast<size_t>(nseg)) +
+              a16(static_cast<size_t>(tok)));
+}
+
+// Checks of the arguments of lora_shrink other than its pointers.
+lora_status shrink_scalar_check(int64_t ld_x, int64_t ld_out, int tok, int K, int S, int r,
+                                int rs, int nseg, int L, lora_dtype dtype, const void* workspace,
+                                size_t workspace_bytes) {
+  if (dtype != LORA_BF16 && dtype != LORA_FP16) return LORA_ERR_UNSUPPORTED;
+  if (tok < 0 || nseg < 0 || K < 1 || S < 1 || r < 1 || rs < r || L < 1)
+    return LORA_ERR_INVALID_ARGUMENT;
+  if (S > LORA_MAX_SLICES) return LORA_ERR_UNSUPPORTED;
+  if (ld_x < K || ld_out < static_cast<int64_t>(S) * rs) return LORA_ERR_INVALID_ARGUMENT;
+  if (workspace_bytes > 0 && !workspace) return LORA_ERR_INVALID_ARGUMENT;
+  return LORA_OK;
+}
+
+// Checks of the arguments of lora_expand other than its device pointers;
+// fills the slice table.
+lora_status expand_scalar_check(int64_t ld_in, int64_t ld_base, int tok, int S, int r, int rs,
+                                int nseg, int L, const int32_t* slice_offsets, lora_dtype dtype,
+                                const void* workspace, size_t workspace_bytes,
+                                lora::SliceTable& tab) {
+  if (dtype != LORA_BF16 && dtype != LORA_FP16) return LORA_ERR_UNSUPPORTED;
+  if (tok < 0 || nseg < 0 || S < 1 || r < 1 || rs < r || L < 1)
+    return LORA_ERR_INVALID_ARGUMENT;
+  if (S > LORA_MAX_SLICES) return LORA_ERR_UNSUPPORTED;
+  if (!slice_offsets) return LORA_ERR_INVALID_ARGUMENT;
+  if (ld_in < static_cast<int64_t>(S) * rs) return LORA_ERR_INVALID_ARGUMENT;
+  if (workspace_bytes > 0 && !workspace) return LORA_ERR_INVALID_ARGUMENT;
+  tab = lora::SliceTable{};
+  tab.S = S;
+  for (int q = 0; q <= S; ++q) {
+    tab.off[q] = slice_offsets[q];
+    if (slice_offsets[q] < 0 || slice_offsets[q] > ld_base) return LORA_ERR_INVALID_ARGUMENT;
+    if (q > 0 && slice_offsets[q] < slice_offsets[q - 1]) return LORA_ERR_INVALID_ARGUMENT;
+  }
+  return LORA_OK;
+}
+
+// Narrows the int64 tables of an *_i64 call into the front of `ws`, at the
+// offsets index64_bytes lays out.
+lora_status narrow_tables(const int64_t* seg_indptr, const int64_t* weight_indices,
+                          const int64_t* permutation, int tok, int nseg, int32_t* ws,
+                          cudaStream_t st) {
+  const int pa = static_cast<int>(a16(static_cast<size_t>(nseg) + 1));
+  const int pb = static_cast<int>(a16(static_cast<size_t>(nseg)));
+  const int nc = permutation ? tok : 0;
+  const int64_t total = static_cast<int64_t>(pa) + pb + nc;
+  const int threads = 256;
+  const unsigned blocks = static_cast<unsigned>((total + threads - 1) / threads);
+  lora::narrow_index_kernel<<<blocks, threads, 0, st>>>(seg_indptr, nseg + 1, pa,
+                                                        weight_indices, nseg, pb,
+                                                        permutation, nc, ws);
+  ++g_launches;
+  return launch_status();
 }
 
 // Enqueues the grouping pass when the schedule calls for it.
@@ -392,6 +473,109 @@ lora_status expand_tc(const lora::ExpandArgs& a, lora_dtype dt, const Grouping& 
   return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ fused shrink + expand
+
+#ifndef LORA_FUSED_MAX_TOK
+#define LORA_FUSED_MAX_TOK 512  // larger batches run the two kernels one after the other
+#endif
+
+// Launches the fused kernel when it applies; *launched says whether it did.
+template <class E>
+lora_status fused_tc(const lora::ShrinkArgs& sa, const lora::ExpandArgs& ea, lora_dtype dt,
+                     const DeviceFacts& dev, cudaStream_t st, bool& launched) {
+  launched = false;
+  if (sa.tok > LORA_FUSED_MAX_TOK) return LORA_OK;
+  lora::FusedTcParams P;
+  std::memset(&P, 0, sizeof(P));
+  P.s = sa;
+  P.e = ea;
+  P.npad = round_up(sa.S * sa.rs, 16);
+  P.nkb = (sa.K + lora::kTcAtomK - 1) / lora::kTcAtomK;
+  P.idesc_s = lora::make_idesc_f16(dt == LORA_BF16 ? 1 : 0, lora::kTcBM, P.npad);
+  P.stage_bytes = lora::kTcBM * 128 + P.npad * 128;
+  P.rpad = ea.r <= 16 ? 16 : (ea.r <= 32 ? 32 : 64);
+  P.sw_layout = P.rpad == 16 ? 6u : (P.rpad == 32 ? 4u : 2u);
+  const CUtensorMapSwizzle swz = P.rpad == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                 : P.rpad == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                : CU_TENSOR_MAP_SWIZZLE_128B;
+  P.rin_bytes = lora::kExBM * P.rpad * 2;
+  P.btile_bytes = lora::kExBN * P.rpad * 2;
+  P.idesc_e = lora::make_idesc_f16(dt == LORA_BF16 ? 1 : 0, lora::kExBM, lora::kExBN);
+  int tiles = 0;
+  for (int q = 0; q < ea.S; ++q) {
+    P.tile_prefix[q] = tiles;
+    tiles += (ea.slices.off[q + 1] - ea.slices.off[q] + lora::kExBN - 1) / lora::kExBN;
+  }
+  for (int q = ea.S; q <= LORA_MAX_SLICES; ++q) P.tile_prefix[q] = tiles;
+  P.tiles_total = tiles;
+  // shared memory: shrink ring (also the split-K partial), rank activations,
+  // base ring, B ring, tokens, barriers; one CTA per SM (the kernel holds all
+  // 512 TMEM columns).  The deepest expand rings that leave room for a shrink
+  // ring of at least two stages holding the partial; otherwise the pair runs
+  // unfused.
+  const size_t part_bytes = sizeof(float) * lora::kTcBM * (P.npad + 4);
+  auto total = [&](int stages) {
+    return static_cast<size_t>(stages) * P.stage_bytes +
+           static_cast<size_t>(sa.S) * P.rin_bytes +
+           static_cast<size_t>(P.base_stages) * lora::kExStageBytes +
+           static_cast<size_t>(P.b_stages) * P.btile_bytes + 1024 + 512 +
+           8 * (2 * stages + 1 + 2 * P.b_stages + 4 + 2 * P.base_stages) + 16;
+  };
+  const int s_min = std::max<int>(2, static_cast<int>((part_bytes + P.stage_bytes - 1) /
+                                                      P.stage_bytes));
+  const int rings[3][2] = {{2, LORA_EXPAND_B_STAGES}, {2, 2}, {1, 2}};  // {base, B}
+  bool fits = false;
+  for (int i = 0; i < 3 && !fits; ++i) {
+    P.base_stages = rings[i][0];
+    P.b_stages = rings[i][1];
+    fits = s_min <= 6 && total(s_min) <= 227 * 1024;
+  }
+  if (!fits) return LORA_OK;
+  P.stages = s_min;
+  while (P.stages < 6 && total(P.stages + 1) <= 227 * 1024) ++P.stages;
+  // at least 120 KB, so that two CTAs never share an SM (and its TMEM)
+  const size_t smem = std::max<size_t>(total(P.stages), 120 * 1024);
+
+  // cluster size: the largest of 16, 8, 4 CTAs for which every expected piece
+  // (one per 128 rows plus about half a piece per segment) gets a resident
+  // cluster and every CTA at least one K block; otherwise the pair runs unfused
+  const long slots = lora::num_piece_slots(sa.tok, sa.nseg, lora::kTcBM);
+  const int est = (sa.tok + lora::kTcBM - 1) / lora::kTcBM + (sa.nseg + 1) / 2;
+  int cs = 0;
+  for (int lg = 4; lg >= 2 && cs == 0; --lg) {
+    const int c = 1 << lg;
+    if (c <= dev.max_cluster && P.nkb >= c && est <= dev.fused_clusters[lg]) cs = c;
+  }
+  if (cs == 0) return LORA_OK;
+  P.csplit = cs;
+
+  const int64_t n_tot = ea.slices.off[ea.S] - ea.slices.off[0];
+  if (!encode_2d(&P.tmap_A, dt, sa.A, sa.K, static_cast<uint64_t>(sa.L) * sa.S * sa.rs,
+                 static_cast<uint64_t>(sa.K) * 2, lora::kTcAtomK, P.npad,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&P.tmap_B, dt, ea.B, ea.r, static_cast<uint64_t>(ea.L) * n_tot,
+                 static_cast<uint64_t>(ea.rs) * 2, P.rpad, lora::kExBN, swz))
+    return LORA_ERR_CUDA;
+
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(static_cast<unsigned>(slots * cs));
+  cfg.blockDim = dim3(lora::kFuThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, lora::fused_tc_kernel<E>, P);
+  ++g_launches;
+  launched = true;
+  g_last_path = LORA_PATH_TENSOR | LORA_PATH_FUSED | LORA_PATH_SPLITK;
+  return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -410,6 +594,11 @@ const char* lora_status_string(lora_status s) {
 uint64_t lora_launch_count(void) { return g_launches; }
 void lora_reset_launch_count(void) { g_launches = 0; }
 int lora_last_path(void) { return g_last_path; }
+
+size_t lora_index64_workspace_size(int tok, int nseg) {
+  if (tok < 0 || nseg < 0) return 0;
+  return index64_bytes(tok, nseg);
+}
 
 size_t lora_workspace_size(int tok, int nseg, int L) {
   if (tok < 0 || nseg < 0 || L < 1) return 0;
@@ -440,12 +629,9 @@ lora_status lora_shrink(const void* x, int64_t ld_x, const void* A_stack,
                         const int32_t* permutation, void* out_r, int64_t ld_out, int tok,
                         int K, int S, int r, int rs, int nseg, int L, lora_dtype dtype,
                         void* workspace, size_t workspace_bytes, void* stream) {
-  if (dtype != LORA_BF16 && dtype != LORA_FP16) return LORA_ERR_UNSUPPORTED;
-  if (tok < 0 || nseg < 0 || K < 1 || S < 1 || r < 1 || rs < r || L < 1)
-    return LORA_ERR_INVALID_ARGUMENT;
-  if (S > LORA_MAX_SLICES) return LORA_ERR_UNSUPPORTED;
-  if (ld_x < K || ld_out < static_cast<int64_t>(S) * rs) return LORA_ERR_INVALID_ARGUMENT;
-  if (workspace_bytes > 0 && !workspace) return LORA_ERR_INVALID_ARGUMENT;
+  const lora_status cs = shrink_scalar_check(ld_x, ld_out, tok, K, S, r, rs, nseg, L, dtype,
+                                             workspace, workspace_bytes);
+  if (cs != LORA_OK) return cs;
   if (tok == 0 || nseg == 0) return LORA_OK;  // nothing to read or write
   if (!x || !A_stack || !seg_indptr || !weight_indices || !out_r)
     return LORA_ERR_INVALID_ARGUMENT;
@@ -479,20 +665,11 @@ lora_status lora_expand(const void* in_r, int64_t ld_in, const void* B_stack,
                         const float* scalings, void* base_out, int64_t ld_base, int tok, int S,
                         int r, int rs, int nseg, int L, lora_dtype dtype, void* workspace,
                         size_t workspace_bytes, void* stream) {
-  if (dtype != LORA_BF16 && dtype != LORA_FP16) return LORA_ERR_UNSUPPORTED;
-  if (tok < 0 || nseg < 0 || S < 1 || r < 1 || rs < r || L < 1)
-    return LORA_ERR_INVALID_ARGUMENT;
-  if (S > LORA_MAX_SLICES) return LORA_ERR_UNSUPPORTED;
-  if (!slice_offsets) return LORA_ERR_INVALID_ARGUMENT;
-  if (ld_in < static_cast<int64_t>(S) * rs) return LORA_ERR_INVALID_ARGUMENT;
-  if (workspace_bytes > 0 && !workspace) return LORA_ERR_INVALID_ARGUMENT;
-  lora::SliceTable tab{};
-  tab.S = S;
-  for (int q = 0; q <= S; ++q) {
-    tab.off[q] = slice_offsets[q];
-    if (slice_offsets[q] < 0 || slice_offsets[q] > ld_base) return LORA_ERR_INVALID_ARGUMENT;
-    if (q > 0 && slice_offsets[q] < slice_offsets[q - 1]) return LORA_ERR_INVALID_ARGUMENT;
-  }
+  lora::SliceTable tab;
+  const lora_status cs = expand_scalar_check(ld_in, ld_base, tok, S, r, rs, nseg, L,
+                                             slice_offsets, dtype, workspace, workspace_bytes,
+                                             tab);
+  if (cs != LORA_OK) return cs;
   if (tok == 0 || nseg == 0 || tab.off[S] == tab.off[0]) return LORA_OK;
   if (!in_r || !B_stack || !seg_indptr || !weight_indices || !scalings || !base_out)
     return LORA_ERR_INVALID_ARGUMENT;
@@ -686,4 +863,133 @@ extern "C" lora_status lora_shrink_static_scratch(
   if (ws == nullptr) return LORA_ERR_CUDA;
   return lora_shrink(x, ld_x, A_stack, seg_indptr, weight_indices, permutation, out_r, ld_out,
                      tok, K, S, r, rs, nseg, L, dtype, ws, LORA_STATIC_SCRATCH_BYTES, stream);
+}
+
+// ------------------------------------------------------------------ int64 index tables
+
+extern "C" lora_status lora_shrink_i64(const void* x, int64_t ld_x, const void* A_stack,
+                                       const int64_t* seg_indptr,
+                                       const int64_t* weight_indices,
+                                       const int64_t* permutation, void* out_r, int64_t ld_out,
+                                       int tok, int K, int S, int r, int rs, int nseg, int L,
+                                       lora_dtype dtype, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  const lora_status cs = shrink_scalar_check(ld_x, ld_out, tok, K, S, r, rs, nseg, L, dtype,
+                                             workspace, workspace_bytes);
+  if (cs != LORA_OK) return cs;
+  if (tok == 0 || nseg == 0) return LORA_OK;
+  // every argument error is reported before the narrowing is enqueued
+  if (!x || !A_stack || !out_r || !aligned_to(x, 2) || !aligned_to(A_stack, 2) ||
+      !aligned_to(out_r, 2))
+    return LORA_ERR_INVALID_ARGUMENT;
+  if (!seg_indptr || !weight_indices || !aligned_to(seg_indptr, 8) ||
+      !aligned_to(weight_indices, 8) || (permutation && !aligned_to(permutation, 8)))
+    return LORA_ERR_INVALID_ARGUMENT;
+  const size_t need = index64_bytes(tok, nseg);
+  if (!workspace || !aligned_to(workspace, 16) || workspace_bytes < need)
+    return LORA_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* w = static_cast<int32_t*>(workspace);
+  const lora_status ns = narrow_tables(seg_indptr, weight_indices, permutation, tok, nseg, w, st);
+  if (ns != LORA_OK) return ns;
+  const int32_t* seg32 = w;
+  const int32_t* wid32 = seg32 + a16(static_cast<size_t>(nseg) + 1);
+  const int32_t* perm32 = permutation ? wid32 + a16(static_cast<size_t>(nseg)) : nullptr;
+  return lora_shrink(x, ld_x, A_stack, seg32, wid32, perm32, out_r, ld_out, tok, K, S, r, rs,
+                     nseg, L, dtype, static_cast<uint8_t*>(workspace) + need,
+                     workspace_bytes - need, stream);
+}
+
+extern "C" lora_status lora_expand_i64(const void* in_r, int64_t ld_in, const void* B_stack,
+                                       const int64_t* seg_indptr,
+                                       const int64_t* weight_indices,
+                                       const int64_t* permutation, const int32_t* slice_offsets,
+                                       const float* scalings, void* base_out, int64_t ld_base,
+                                       int tok, int S, int r, int rs, int nseg, int L,
+                                       lora_dtype dtype, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  lora::SliceTable tab;
+  const lora_status cs = expand_scalar_check(ld_in, ld_base, tok, S, r, rs, nseg, L,
+                                             slice_offsets, dtype, workspace, workspace_bytes,
+                                             tab);
+  if (cs != LORA_OK) return cs;
+  if (tok == 0 || nseg == 0 || tab.off[S] == tab.off[0]) return LORA_OK;
+  // every argument error is reported before the narrowing is enqueued
+  if (!in_r || !B_stack || !scalings || !base_out || !aligned_to(in_r, 2) ||
+      !aligned_to(B_stack, 2) || !aligned_to(scalings, 4) || !aligned_to(base_out, 2))
+    return LORA_ERR_INVALID_ARGUMENT;
+  if (!seg_indptr || !weight_indices || !aligned_to(seg_indptr, 8) ||
+      !aligned_to(weight_indices, 8) || (permutation && !aligned_to(permutation, 8)))
+    return LORA_ERR_INVALID_ARGUMENT;
+  const size_t need = index64_bytes(tok, nseg);
+  if (!workspace || !aligned_to(workspace, 16) || workspace_bytes < need)
+    return LORA_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* w = static_cast<int32_t*>(workspace);
+  const lora_status ns = narrow_tables(seg_indptr, weight_indices, permutation, tok, nseg, w, st);
+  if (ns != LORA_OK) return ns;
+  const int32_t* seg32 = w;
+  const int32_t* wid32 = seg32 + a16(static_cast<size_t>(nseg) + 1);
+  const int32_t* perm32 = permutation ? wid32 + a16(static_cast<size_t>(nseg)) : nullptr;
+  return lora_expand(in_r, ld_in, B_stack, seg32, wid32, perm32, slice_offsets, scalings,
+                     base_out, ld_base, tok, S, r, rs, nseg, L, dtype,
+                     static_cast<uint8_t*>(workspace) + need, workspace_bytes - need, stream);
+}
+
+// ------------------------------------------------------------------ fused pair
+
+extern "C" lora_status lora_shrink_expand(
+    const void* x, int64_t ld_x, const void* A_stack, const void* B_stack,
+    const int32_t* seg_indptr, const int32_t* weight_indices, const int32_t* permutation,
+    const int32_t* slice_offsets, const float* scalings, void* out_r, int64_t ld_out,
+    void* base_out, int64_t ld_base, int tok, int K, int S, int r, int rs, int nseg, int L,
+    lora_dtype dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  const lora_status cs = shrink_scalar_check(ld_x, ld_out, tok, K, S, r, rs, nseg, L, dtype,
+                                             workspace, workspace_bytes);
+  if (cs != LORA_OK) return cs;
+  lora::SliceTable tab;
+  const lora_status ce = expand_scalar_check(ld_out, ld_base, tok, S, r, rs, nseg, L,
+                                             slice_offsets, dtype, workspace, workspace_bytes,
+                                             tab);
+  if (ce != LORA_OK) return ce;
+  if (tok == 0 || nseg == 0) return LORA_OK;
+  if (!x || !A_stack || !B_stack || !seg_indptr || !weight_indices || !scalings || !out_r ||
+      !base_out)
+    return LORA_ERR_INVALID_ARGUMENT;
+  if (!aligned_to(x, 2) || !aligned_to(A_stack, 2) || !aligned_to(B_stack, 2) ||
+      !aligned_to(out_r, 2) || !aligned_to(base_out, 2) || !aligned_to(seg_indptr, 4) ||
+      !aligned_to(weight_indices, 4) || !aligned_to(scalings, 4) ||
+      (permutation && !aligned_to(permutation, 4)))
+    return LORA_ERR_INVALID_ARGUMENT;
+
+  const lora::ShrinkArgs sa{static_cast<const uint16_t*>(x), ld_x,
+                            static_cast<const uint16_t*>(A_stack), seg_indptr, weight_indices,
+                            permutation, static_cast<uint16_t*>(out_r), ld_out, tok, K, S, r,
+                            rs, nseg, L};
+  const lora::ExpandArgs ea{static_cast<const uint16_t*>(out_r), ld_out,
+                            static_cast<const uint16_t*>(B_stack), seg_indptr, weight_indices,
+                            permutation, scalings, static_cast<uint16_t*>(base_out), ld_base,
+                            tok, S, r, rs, nseg, L, tab};
+  const DeviceFacts* dev = device_facts();
+  if (!dev) return LORA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (shrink_tc_eligible(sa) && expand_tc_eligible(ea) && tab.off[S] > tab.off[0]) {
+    bool launched = false;
+    const lora_status fs = dtype == LORA_BF16
+                               ? fused_tc<lora::Bf16>(sa, ea, dtype, *dev, st, launched)
+                               : fused_tc<lora::Fp16>(sa, ea, dtype, *dev, st, launched);
+    if (fs != LORA_OK || launched) return fs;
+  }
+  // the composition: the shrink's rounded output is the expand's input
+  const lora_status s1 = lora_shrink(x, ld_x, A_stack, seg_indptr, weight_indices, permutation,
+                                     out_r, ld_out, tok, K, S, r, rs, nseg, L, dtype, workspace,
+                                     workspace_bytes, stream);
+  if (s1 != LORA_OK) return s1;
+  const int path = g_last_path;
+  const lora_status s2 = lora_expand(out_r, ld_out, B_stack, seg_indptr, weight_indices,
+                                     permutation, slice_offsets, scalings, base_out, ld_base,
+                                     tok, S, r, rs, nseg, L, dtype, workspace, workspace_bytes,
+                                     stream);
+  g_last_path |= path;
+  return s2;
 }

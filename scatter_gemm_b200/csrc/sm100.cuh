@@ -277,6 +277,18 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
   return r;
 }
 
+// 8-byte store into the shared memory of a CTA of this cluster (address from mapa)
+__device__ __forceinline__ void st_dsmem_v2(uint32_t caddr, uint32_t lo, uint32_t hi) {
+  asm volatile("st.shared::cluster.v2.b32 [%0], {%1, %2};" ::"r"(caddr), "r"(lo), "r"(hi)
+               : "memory");
+}
+
+// Orders this thread's earlier generic-proxy writes, in every state space
+// (including other CTAs' shared memory), before later async-proxy accesses.
+__device__ __forceinline__ void fence_proxy_async_all() {
+  asm volatile("fence.proxy.async;" ::: "memory");
+}
+
 __device__ __forceinline__ float4 ld_dsmem_v4(uint32_t caddr) {
   float4 v;
   asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"

@@ -65,6 +65,15 @@ def lib() -> ctypes.CDLL:
             l.lora_last_path.restype = _I
             l.lora_device_error.argtypes = [_P, _I]
             l.lora_device_error.restype = _I
+            l.lora_shrink_i64.argtypes = l.lora_shrink.argtypes
+            l.lora_shrink_i64.restype = _I
+            l.lora_expand_i64.argtypes = l.lora_expand.argtypes
+            l.lora_expand_i64.restype = _I
+            l.lora_index64_workspace_size.argtypes = [_I, _I]
+            l.lora_index64_workspace_size.restype = _Z
+            l.lora_shrink_expand.argtypes = [_P, _L, _P, _P, _P, _P, _P, _P, _P, _P, _L, _P, _L] + \
+                [_I] * 8 + [_P, _Z, _P]
+            l.lora_shrink_expand.restype = _I
             _lib = l
     return _lib
 
@@ -81,7 +90,7 @@ def reset_launch_count() -> None:
     lib().lora_reset_launch_count()
 
 
-PATH_GENERAL, PATH_TENSOR, PATH_GROUPED, PATH_SPLITK = 1, 2, 4, 8
+PATH_GENERAL, PATH_TENSOR, PATH_GROUPED, PATH_SPLITK, PATH_FUSED = 1, 2, 4, 8, 16
 
 
 def last_path() -> int:
@@ -125,14 +134,37 @@ def _row_major(t: torch.Tensor, name: str, dims: int = 2) -> int:
     return t.stride(0) if dims == 2 else 0
 
 
-def _table(t: Optional[torch.Tensor], name: str, allow_none: bool = False):
+def _table(t: Optional[torch.Tensor], name: str, allow_none: bool = False,
+           dtype: torch.dtype = torch.int32):
     if t is None:
         if allow_none:
             return None
         raise ValueError(f"{name} is required")
-    if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
-        raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+    if t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} CUDA tensor")
     return t.data_ptr()
+
+
+def _index_dtype(*tables: Optional[torch.Tensor]) -> torch.dtype:
+    """int32 or int64: the one index type all given tables share."""
+    kinds = {t.dtype for t in tables if t is not None}
+    if len(kinds) != 1 or not kinds <= {torch.int32, torch.int64}:
+        raise ValueError("index tables must all be int32 or all be int64")
+    return kinds.pop()
+
+
+def index64_workspace_size(tok: int, nseg: int) -> int:
+    """Bytes at the front of an int64-table call's workspace (the narrowed tables)."""
+    return int(lib().lora_index64_workspace_size(tok, nseg))
+
+
+def _ws64(workspace: Optional[torch.Tensor], tok: int, nseg: int, num_adapters: int, device):
+    """Workspace of an int64-table call: the caller's, or one allocated here
+    (narrowed tables followed by the adapter-grouping scratch)."""
+    if workspace is None:
+        n = index64_workspace_size(tok, nseg) + workspace_size(tok, nseg, num_adapters)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+    return workspace, _ws(workspace)
 
 
 def _stream(stream) -> int:
@@ -157,7 +189,9 @@ def lora_shrink(x: torch.Tensor, A_stack: torch.Tensor, seg_indptr: torch.Tensor
 
     x [tok, K] (unit inner stride), A_stack [L, S*rs, K] contiguous (or
     [L, S, rs, K]), out_r [tok, >= S*rs] (unit inner stride, sorted order).
-    `rank` is the valid rank r <= rs (default rs)."""
+    `rank` is the valid rank r <= rs (default rs).  The index tables are all
+    int32, or all int64 (then lora_shrink_i64 runs, and a workspace is
+    allocated when none is given)."""
     dt = _dtype_code(x)
     if A_stack.dtype != x.dtype or out_r.dtype != x.dtype:
         raise TypeError("x, A_stack and out_r must share one element type")
@@ -184,13 +218,20 @@ def lora_shrink(x: torch.Tensor, A_stack: torch.Tensor, seg_indptr: torch.Tensor
     if out_r.shape[0] != tok:
         raise ValueError("out_r must have one row per token")
     nseg = seg_indptr.numel() - 1
-    ws, wsb = _ws(workspace)
-    st = lib().lora_shrink(x.data_ptr(), ld_x, A_stack.data_ptr(),
-                           _table(seg_indptr, "seg_indptr"), _table(weight_indices, "weight_indices"),
-                           _table(permutation, "permutation", True), out_r.data_ptr(), ld_out,
-                           tok, K, S, r, rs, nseg, L, dt, ws, wsb, _stream(stream))
+    idt = _index_dtype(seg_indptr, weight_indices, permutation)
+    if idt == torch.int64:
+        # int64 tables: lora_shrink_i64 narrows them into the workspace first
+        workspace, (ws, wsb) = _ws64(workspace, tok, nseg, L, x.device)
+        fn, name = lib().lora_shrink_i64, "lora_shrink_i64"
+    else:
+        ws, wsb = _ws(workspace)
+        fn, name = lib().lora_shrink, "lora_shrink"
+    st = fn(x.data_ptr(), ld_x, A_stack.data_ptr(), _table(seg_indptr, "seg_indptr", dtype=idt),
+            _table(weight_indices, "weight_indices", dtype=idt),
+            _table(permutation, "permutation", True, dtype=idt), out_r.data_ptr(), ld_out,
+            tok, K, S, r, rs, nseg, L, dt, ws, wsb, _stream(stream))
     if st != LORA_OK:
-        raise LoraError("lora_shrink", st)
+        raise LoraError(name, st)
     return out_r
 
 
@@ -203,7 +244,8 @@ def lora_expand(in_r: torch.Tensor, B_stack: torch.Tensor, seg_indptr: torch.Ten
 
     in_r [tok, >= S*rs] (sorted order), B_stack [L, N_tot, rs] contiguous,
     slice_offsets: S+1 host integers, scalings [L] fp32 CUDA, base_out
-    [tok, >= off[S]] updated in place."""
+    [tok, >= off[S]] updated in place.  Index tables: all int32, or all int64
+    (lora_expand_i64, as for lora_shrink)."""
     dt = _dtype_code(base_out)
     if in_r.dtype != base_out.dtype or B_stack.dtype != base_out.dtype:
         raise TypeError("in_r, B_stack and base_out must share one element type")
@@ -227,15 +269,76 @@ def lora_expand(in_r: torch.Tensor, B_stack: torch.Tensor, seg_indptr: torch.Ten
         raise ValueError("in_r must have one row per token")
     nseg = seg_indptr.numel() - 1
     off_arr = (ctypes.c_int32 * len(off))(*off)
-    ws, wsb = _ws(workspace)
-    st = lib().lora_expand(in_r.data_ptr(), ld_in, B_stack.data_ptr(),
-                           _table(seg_indptr, "seg_indptr"), _table(weight_indices, "weight_indices"),
-                           _table(permutation, "permutation", True),
-                           ctypes.cast(off_arr, ctypes.c_void_p), scalings.data_ptr(),
-                           base_out.data_ptr(), ld_base, tok, S, r, rs, nseg, L, dt, ws, wsb,
-                           _stream(stream))
+    idt = _index_dtype(seg_indptr, weight_indices, permutation)
+    if idt == torch.int64:
+        # int64 tables: lora_expand_i64 narrows them into the workspace first
+        workspace, (ws, wsb) = _ws64(workspace, tok, nseg, L, base_out.device)
+        fn, name = lib().lora_expand_i64, "lora_expand_i64"
+    else:
+        ws, wsb = _ws(workspace)
+        fn, name = lib().lora_expand, "lora_expand"
+    st = fn(in_r.data_ptr(), ld_in, B_stack.data_ptr(),
+            _table(seg_indptr, "seg_indptr", dtype=idt),
+            _table(weight_indices, "weight_indices", dtype=idt),
+            _table(permutation, "permutation", True, dtype=idt),
+            ctypes.cast(off_arr, ctypes.c_void_p), scalings.data_ptr(),
+            base_out.data_ptr(), ld_base, tok, S, r, rs, nseg, L, dt, ws, wsb,
+            _stream(stream))
     if st != LORA_OK:
-        raise LoraError("lora_expand", st)
+        raise LoraError(name, st)
+    return base_out
+
+
+def lora_shrink_expand(x: torch.Tensor, A_stack: torch.Tensor, B_stack: torch.Tensor,
+                       seg_indptr: torch.Tensor, weight_indices: torch.Tensor,
+                       permutation: Optional[torch.Tensor], slice_offsets: Sequence[int],
+                       scalings: torch.Tensor, out_r: torch.Tensor, base_out: torch.Tensor, *,
+                       rank: Optional[int] = None, workspace: Optional[torch.Tensor] = None,
+                       stream=None) -> torch.Tensor:
+    """The pair in one call: lora_shrink into out_r, then lora_expand of out_r
+    into base_out (one fused launch for decode-sized batches).
+
+    x [tok, K], A_stack [L, S*rs, K], B_stack [L, N_tot, rs], out_r
+    [tok, >= S*rs] (written), base_out [tok, >= off[S]] (updated), int32 tables."""
+    dt = _dtype_code(x)
+    for t, n in ((A_stack, "A_stack"), (B_stack, "B_stack"), (out_r, "out_r"),
+                 (base_out, "base_out")):
+        if t.dtype != x.dtype:
+            raise TypeError(f"{n} must have the element type of x")
+    if scalings.dtype != torch.float32 or not scalings.is_cuda or not scalings.is_contiguous():
+        raise ValueError("scalings must be a contiguous fp32 CUDA tensor")
+    ld_x = _row_major(x, "x")
+    ld_out = _row_major(out_r, "out_r")
+    ld_base = _row_major(base_out, "base_out")
+    if not A_stack.is_contiguous() or A_stack.dim() != 3:
+        raise ValueError("A_stack must be a contiguous [L, S*rs, K] tensor")
+    if B_stack.dim() != 3 or not B_stack.is_contiguous():
+        raise ValueError("B_stack must be a contiguous [L, N_tot, rs] tensor")
+    L, srs, K = A_stack.shape
+    Lb, n_tot, rs = B_stack.shape
+    off = [int(v) for v in (slice_offsets.tolist() if torch.is_tensor(slice_offsets)
+                            else slice_offsets)]
+    S = len(off) - 1
+    if S < 1 or S > MAX_SLICES or srs != S * rs or Lb != L:
+        raise ValueError("A_stack, B_stack and slice_offsets disagree on L, S or rs")
+    if off[-1] - off[0] != n_tot:
+        raise ValueError("slice_offsets span does not match B_stack rows")
+    tok, Kx = x.shape
+    if Kx != K or out_r.shape[0] != tok or base_out.shape[0] != tok:
+        raise ValueError("x, out_r and base_out must have one row per token and K columns")
+    r = rs if rank is None else int(rank)
+    nseg = seg_indptr.numel() - 1
+    off_arr = (ctypes.c_int32 * len(off))(*off)
+    ws, wsb = _ws(workspace)
+    st = lib().lora_shrink_expand(x.data_ptr(), ld_x, A_stack.data_ptr(), B_stack.data_ptr(),
+                                  _table(seg_indptr, "seg_indptr"),
+                                  _table(weight_indices, "weight_indices"),
+                                  _table(permutation, "permutation", True),
+                                  ctypes.cast(off_arr, ctypes.c_void_p), scalings.data_ptr(),
+                                  out_r.data_ptr(), ld_out, base_out.data_ptr(), ld_base, tok,
+                                  K, S, r, rs, nseg, L, dt, ws, wsb, _stream(stream))
+    if st != LORA_OK:
+        raise LoraError("lora_shrink_expand", st)
     return base_out
 
 

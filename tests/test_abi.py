@@ -105,6 +105,85 @@ def test_expand_rejects_bad_slice_tables(L):
     assert expand(L, off=(8, 8), S=1, tok=5) == OK        # no columns: nothing to do
 
 
+def shrink64(lib, **kw):
+    a = dict(x=P, ld_x=64, A=P, si=P, wi=P, pm=P, out=P, ld_out=48, tok=10, K=64, S=3, r=16,
+             rs=16, nseg=2, nad=4, dt=0, ws=P, wsb=1 << 20, st=None)
+    a.update(kw)
+    return lib.lora_shrink_i64(a["x"], a["ld_x"], a["A"], a["si"], a["wi"], a["pm"], a["out"],
+                               a["ld_out"], a["tok"], a["K"], a["S"], a["r"], a["rs"],
+                               a["nseg"], a["nad"], a["dt"], a["ws"], a["wsb"], a["st"])
+
+
+def expand64(lib, off=(0, 32, 40, 48), **kw):
+    arr = (ctypes.c_int32 * len(off))(*off)
+    a = dict(inr=P, ld_in=48, B=P, si=P, wi=P, pm=P, offp=ctypes.cast(arr, ctypes.c_void_p),
+             sc=P, base=P, ld_base=48, tok=10, S=len(off) - 1, r=16, rs=16, nseg=2, nad=4, dt=0,
+             ws=P, wsb=1 << 20, st=None)
+    a.update(kw)
+    return lib.lora_expand_i64(a["inr"], a["ld_in"], a["B"], a["si"], a["wi"], a["pm"],
+                               a["offp"], a["sc"], a["base"], a["ld_base"], a["tok"], a["S"],
+                               a["r"], a["rs"], a["nseg"], a["nad"], a["dt"], a["ws"], a["wsb"],
+                               a["st"])
+
+
+# every case returns before the narrowing kernel would be enqueued
+@pytest.mark.parametrize("kw,want", [
+    (dict(si=None), INVALID), (dict(wi=None), INVALID),
+    (dict(si=P + 4), INVALID), (dict(wi=P + 4), INVALID), (dict(pm=P + 4), INVALID),
+    (dict(ws=None, wsb=0), INVALID),     # the narrowed tables need a workspace
+    (dict(wsb=16), INVALID),             # too small for them
+    (dict(ws=P + 8), INVALID),           # not 16-byte aligned
+    (dict(x=None), INVALID), (dict(out=P + 1), INVALID),
+    (dict(tok=-1), INVALID), (dict(dt=2), UNSUPPORTED), (dict(rs=8), INVALID),
+    (dict(tok=0), OK), (dict(nseg=0), OK),
+])
+def test_shrink_i64_argument_checks(L, kw, want):
+    assert shrink64(L, **kw) == want
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(si=None), INVALID), (dict(pm=P + 4), INVALID), (dict(ws=None, wsb=0), INVALID),
+    (dict(wsb=8), INVALID), (dict(sc=None), INVALID), (dict(base=P + 1), INVALID),
+    (dict(offp=None), INVALID), (dict(dt=3), UNSUPPORTED), (dict(tok=0), OK),
+])
+def test_expand_i64_argument_checks(L, kw, want):
+    assert expand64(L, **kw) == want
+
+
+def pair(lib, off=(0, 32, 40, 48), **kw):
+    arr = (ctypes.c_int32 * len(off))(*off)
+    a = dict(x=P, ld_x=64, A=P, B=P, si=P, wi=P, pm=P, offp=ctypes.cast(arr, ctypes.c_void_p),
+             sc=P, out=P, ld_out=48, base=P, ld_base=48, tok=10, K=64, S=len(off) - 1, r=16,
+             rs=16, nseg=2, nad=4, dt=0, ws=None, wsb=0, st=None)
+    a.update(kw)
+    return lib.lora_shrink_expand(a["x"], a["ld_x"], a["A"], a["B"], a["si"], a["wi"], a["pm"],
+                                  a["offp"], a["sc"], a["out"], a["ld_out"], a["base"],
+                                  a["ld_base"], a["tok"], a["K"], a["S"], a["r"], a["rs"],
+                                  a["nseg"], a["nad"], a["dt"], a["ws"], a["wsb"], a["st"])
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(x=None), INVALID), (dict(A=None), INVALID), (dict(B=None), INVALID),
+    (dict(si=None), INVALID), (dict(wi=None), INVALID), (dict(sc=None), INVALID),
+    (dict(out=None), INVALID), (dict(base=None), INVALID), (dict(offp=None), INVALID),
+    (dict(K=0), INVALID), (dict(rs=8), INVALID), (dict(dt=2), UNSUPPORTED),
+    (dict(ld_out=47), INVALID), (dict(ld_base=47), INVALID), (dict(ld_x=63), INVALID),
+    (dict(B=P + 1), INVALID), (dict(sc=P + 2), INVALID), (dict(pm=P + 2), INVALID),
+    (dict(wsb=16), INVALID),
+    (dict(tok=0), OK), (dict(nseg=0), OK),
+])
+def test_shrink_expand_argument_checks(L, kw, want):
+    assert pair(L, **kw) == want
+
+
+def test_index64_workspace_size(L):
+    # narrowed seg_indptr, weight_indices and permutation, each padded to 16 bytes
+    assert lora.index64_workspace_size(100, 3) == 4 * (4 + 4 + 100)
+    assert lora.index64_workspace_size(0, 0) == 16
+    assert lora.index64_workspace_size(7, 5) == 4 * (8 + 8 + 8)
+    assert L.lora_index64_workspace_size(-1, 2) == 0
+
+
 def test_workspace_sizes(L):
     assert lora.workspace_size(0, 0, 1) > 0
     assert lora.workspace_size(8192, 1024, 64) >= 4 * (8192 + 65)
