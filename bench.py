@@ -160,6 +160,7 @@ class DevProblem:
         self.ws = lora.make_workspace(p.tok, p.nseg, p.L, device)
         self.bytes_shrink = W.bytes_shrink(p)
         self.bytes_expand = W.bytes_expand(p)
+        self.rows = int(p.seg_indptr[-1] - p.seg_indptr[0])
 
     def shrink(self, lora):
         lora.lora_shrink(self.x, self.A, self.si, self.wi, self.pm, self.out,
@@ -168,6 +169,40 @@ class DevProblem:
     def expand(self, lora):
         lora.lora_expand(self.out, self.B, self.si, self.wi, self.pm, self.off, self.sc,
                          self.base, rank=self.p.r, workspace=self.ws)
+
+    def pair(self, lora):
+        lora.lora_shrink_expand(self.x, self.A, self.B, self.si, self.wi, self.pm, self.off,
+                                self.sc, self.out, self.base, rank=self.p.r, workspace=self.ws)
+
+
+def time_fused(probs, lora, flush, stream, steps, warmup, nap):
+    """lora_shrink_expand on the decode-sized cases of the sweep (tok <= 512),
+    timed like the sweep: L2 flushed and a GPU sleep before each call, CUDA
+    events around it.  Reported beside the separately timed pair, not part of
+    `value` (the pages measure the two ops one by one)."""
+    out = []
+    for dp in probs:
+        if dp.p.tok > 512:
+            continue
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for k in range(warmup + steps):
+            flush.zero_()
+            torch.cuda._sleep(nap)
+            if k >= warmup:
+                ev[k - warmup][0].record(stream)
+            dp.pair(lora)
+            if k >= warmup:
+                ev[k - warmup][1].record(stream)
+        torch.cuda.synchronize()
+        ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+        # algorithmic bytes of the fused call: both ops' bytes less the rank
+        # activations the expand would read back
+        nbytes = dp.bytes_shrink + dp.bytes_expand - dp.rows * dp.p.S * dp.p.r * 2
+        out.append({"tok": dp.p.tok, "fused_us": round(ms * 1e3, 2),
+                    "fused_path": bool(lora.last_path() & lora.PATH_FUSED),
+                    "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)})
+    return out
 
 
 # ----------------------------------------------------------------------------
@@ -299,6 +334,9 @@ def run_ours(args, rank, world, device):
         kernel_ms, wall_ms = float(red[0]), float(red[1])
 
     # e2e: host buffers in pinned memory, H2D + both calls + D2H inside the timed region
+    fused = None
+    if not args.no_fused:
+        fused = time_fused(probs, lora, flush, stream, min(args.steps, 200), 3, nap)
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, probs, lora, device, stream, world)
@@ -325,6 +363,12 @@ def run_ours(args, rank, world, device):
         if dp.p.tok >= 1024:
             fr.append(gbs)
     geo = math.exp(sum(math.log(v) for v in fr) / len(fr)) if fr else None
+    if fused:
+        pair = {d["tok"]: d["shrink_us"] + d["expand_us"] for d in detail}
+        for f in fused:
+            if f["tok"] in pair:
+                f["pair_us"] = round(pair[f["tok"]], 2)
+                f["speedup_vs_pair"] = round(pair[f["tok"]] / f["fused_us"], 2)
     mean_case = statistics.mean(d["gbs"] for d in detail)
 
     # roofline of the dominant kernel (larger summed time of the two ops)
@@ -369,6 +413,7 @@ def run_ours(args, rank, world, device):
         "geomean_frac_nominal_tok_ge_1024": round(geo / NOMINAL_HBM_GBS, 4) if geo else None,
         "mean_case_gbs": round(mean_case, 1),
         "per_tok": detail,
+        "fused_decode": fused,
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -435,6 +480,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-fused", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -209,12 +209,11 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
       const int u = j * kExBM + pt;
       const int row = u / kExCh, c = u % kExCh;
       const int col = c0 + 8 * c;
-      const bool in = row < rows && col < cend;
-      cp_async_16(stage + row * (kExBN * 2) + ((c ^ (row & (kExCh - 1))) << 4),
-                  in ? static_cast<const void*>(p.base +
-                                                static_cast<int64_t>(trow[row]) * p.ld_base + col)
-                     : static_cast<const void*>(p.base),
-                  in ? 16u : 0u);
+      // rows past the piece and columns past the slice are not loaded: the
+      // epilogue never stores them
+      if (row < rows && col < cend)
+        cp_async_16(stage + row * (kExBN * 2) + ((c ^ (row & (kExCh - 1))) << 4),
+                    p.base + static_cast<int64_t>(trow[row]) * p.ld_base + col, 16u);
     }
   };
   const int pre = min(P.base_stages, ntl);  // tiles issued before the CTA barrier
@@ -243,8 +242,11 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
         const uint32_t nb = row_ok ? static_cast<uint32_t>(max(0, min(left, 8)) * 2) : 0u;
         const uint32_t dst = rin + q * P.rin_bytes + m * (P.rpad * 2) +
                              (swz_chunk(c, m, P.rpad) << 4);
-        cp_async_16(dst, nb ? static_cast<const void*>(src0 + q * p.rs + 8 * c)
-                            : static_cast<const void*>(p.in_r), nb);
+        // rows past the piece are not loaded (their accumulator rows are never
+        // stored); a row of the piece is zero-filled beyond r
+        if (row_ok)
+          cp_async_16(dst, nb ? static_cast<const void*>(src0 + q * p.rs + 8 * c)
+                              : static_cast<const void*>(p.in_r), nb);
       }
     }
     cp_async_commit();

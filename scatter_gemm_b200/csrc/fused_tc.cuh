@@ -25,8 +25,9 @@
 //   warp 0      TMEM (512 columns: shrink accumulator at column 0, the expand's
 //               double-buffered accumulator at column 256); A and B tiles by
 //               TMA; every MMA;
-//   warps 1-8   expand epilogue (as in expand_tc); warps 1-4 also read the
-//               shrink accumulator out into the split-K partial;
+//   warps 1-8   expand epilogue as two groups of four warps taking alternate
+//               tiles (group g uses accumulator buffer g); warps 1-4 also read
+//               the shrink accumulator out into the split-K partial;
 //   warps 9-12  x gather of the shrink, base tiles of the expand.
 // All threads take part in step 2.
 #pragma once
@@ -43,6 +44,7 @@ namespace lora {
 constexpr int kFuThreads = 416;
 constexpr int kFuTmemCols = 512;
 constexpr int kFuExpandCol = 256;  // first TMEM column of the expand accumulators
+constexpr int kFuGroup = 128;      // threads of one consumer group (four warps)
 
 struct FusedTcParams {
   CUtensorMap tmap_A;  // 2-D [L*S*rs rows, K cols], box {64, NPAD}, 128B swizzle
@@ -62,7 +64,9 @@ struct FusedTcParams {
   uint32_t idesc_e;    // expand: M = 128, N = 128
   int tiles_total;
   int tile_prefix[LORA_MAX_SLICES + 1];
-  int base_stages;
+  int base_stages;     // expand ring stages of their own
+  int xstages;         // expand ring stages in all: the rest live in the shrink ring,
+                       // free once step 2 is over
   int b_stages;
 };
 
@@ -98,9 +102,15 @@ fused_tc_kernel(const __grid_constant__ FusedTcParams P) {
   const uint32_t tfull0 = bempty0 + 8 * P.b_stages;
   const uint32_t tempty0 = tfull0 + 16;
   const uint32_t xfull0 = tempty0 + 16;
-  const uint32_t xempty0 = xfull0 + 8 * P.base_stages;
+  const uint32_t xempty0 = xfull0 + 8 * P.xstages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * P.stages + 1 + 2 * P.b_stages +
-                                                    4 + 2 * P.base_stages);
+                                                    4 + 2 * P.xstages);
+  // expand ring stage s: the first base_stages are the CTA's own, the others
+  // reuse the shrink ring after step 2
+  auto xstage = [&](int s) {
+    return s < P.base_stages ? base_ring + s * kExStageBytes
+                             : ring + (s - P.base_stages) * kExStageBytes;
+  };
 
   if (tid == 32) {
     for (int s = 0; s < P.stages; ++s) {
@@ -114,11 +124,11 @@ fused_tc_kernel(const __grid_constant__ FusedTcParams P) {
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull0 + 8 * b, 1);
-      mbar_init(tempty0 + 8 * b, kExConsumers);
+      mbar_init(tempty0 + 8 * b, kFuGroup);  // accumulator buffer b: consumer group b
     }
-    for (int s = 0; s < P.base_stages; ++s) {
+    for (int s = 0; s < P.xstages; ++s) {
       mbar_init(xfull0 + 8 * s, kExProducers);
-      mbar_init(xempty0 + 8 * s, kExConsumers);
+      mbar_init(xempty0 + 8 * s, kFuGroup);  // released by the group that used the stage
     }
     fence_mbar_init();
   }
@@ -192,19 +202,17 @@ fused_tc_kernel(const __grid_constant__ FusedTcParams P) {
     int q, c0;
     tile_cols(t, q, c0);
     const int cend = pe.slices.off[q + 1];
-    const uint32_t stage = base_ring + s * kExStageBytes;
+    const uint32_t stage = xstage(s);
 #pragma unroll 4
     for (int j = 0; j < kExCh; ++j) {
       const int u = j * kExBM + pt;
       const int row = u / kExCh, c = u % kExCh;
       const int col = c0 + 8 * c;
-      const bool in = row < rows && col < cend;
-      cp_async_16(stage + row * (kExBN * 2) + ((c ^ (row & (kExCh - 1))) << 4),
-                  in ? static_cast<const void*>(pe.base +
-                                                static_cast<int64_t>(trow[row]) * pe.ld_base +
-                                                col)
-                     : static_cast<const void*>(pe.base),
-                  in ? 16u : 0u);
+      // rows past the piece and columns past the slice are not loaded: the
+      // epilogue never stores them
+      if (row < rows && col < cend)
+        cp_async_16(stage + row * (kExBN * 2) + ((c ^ (row & (kExCh - 1))) << 4),
+                    pe.base + static_cast<int64_t>(trow[row]) * pe.ld_base + col, 16u);
     }
   };
   auto load_b = [&](int t, int sp) {
@@ -246,11 +254,14 @@ fused_tc_kernel(const __grid_constant__ FusedTcParams P) {
       const bool k_in = k < ps.K;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
+        // rows past the piece are not loaded (their MMA rows are never used);
+        // past K a row of the piece is zero-filled
         const int row = rr + 16 * j;
-        const bool in = k_in && row < rows;
-        cp_async_16(xs + row * 128 + ((cc ^ (row & 7)) << 4),
-                    in ? static_cast<const void*>(xr[j] + k) : static_cast<const void*>(ps.x),
-                    in ? 16u : 0u);
+        if (row < rows)
+          cp_async_16(xs + row * 128 + ((cc ^ (row & 7)) << 4),
+                      k_in ? static_cast<const void*>(xr[j] + k)
+                           : static_cast<const void*>(ps.x),
+                      k_in ? 16u : 0u);
       }
       cp_async_commit();
       if (i >= lag) {
@@ -403,9 +414,10 @@ fused_tc_kernel(const __grid_constant__ FusedTcParams P) {
     }
     __syncwarp();
   } else if (producer) {
+    // stages of the shrink ring are fresh now: they are filled without waiting
     for (int t = pre_e; t < ntl && ok; ++t) {
-      const int s = t % P.base_stages;
-      ok = mbar_wait(xempty0 + 8 * s, ((t / P.base_stages) - 1) & 1);
+      const int s = t % P.xstages;
+      if (t >= P.xstages) ok = mbar_wait(xempty0 + 8 * s, ((t / P.xstages) - 1) & 1);
       if (!ok) break;
       issue_tile(t, s);
       cp_async_arrive_noinc(xfull0 + 8 * s);
@@ -413,36 +425,37 @@ fused_tc_kernel(const __grid_constant__ FusedTcParams P) {
     }
     cp_async_wait<0>();
   } else {
-    // consumers (warps 1-8), as in expand_tc
+    // consumers: two groups of four warps (one per TMEM lane quarter) take
+    // alternate tiles, so two tiles are in their epilogue at once; group g
+    // uses accumulator buffer g
     const int quarter = warp & 3;
-    const int half = (warp - 1) >> 2;
-    const int m = quarter * 32 + lane;
-    const int ct = tid - 32;
-    for (int t = 0; t < ntl; ++t) {
-      const int s = t % P.base_stages, buf = t & 1;
-      if (ok) ok = mbar_wait(xfull0 + 8 * s, (t / P.base_stages) & 1);
+    const int grp = (warp - 1) >> 2;
+    const int m = quarter * 32 + lane;  // accumulator row of this thread
+    const int gt = tid - 32 - grp * kFuGroup;  // 0..127 in the group
+    for (int t = grp; t < ntl; t += 2) {
+      const int s = t % P.xstages, buf = grp;
+      if (ok) ok = mbar_wait(xfull0 + 8 * s, (t / P.xstages) & 1);
       if (ok) ok = mbar_wait(tfull0 + 8 * buf, (t >> 1) & 1);
-      ok = __all_sync(0xffffffffu, ok);
+      ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
       tc_fence_after();
       int q, c0;
       tile_cols(t, q, c0);
-      uint8_t* stage_p = smem + (base_ring - sbase) + s * kExStageBytes;
+      uint8_t* stage_p = smem + (xstage(s) - sbase);
       const uint32_t tacc = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kFuExpandCol +
                             buf * kExBN;
-      constexpr int kHalfChunks = kExBN / 32;
+      // (a) row m, every column: base + scaling * acc, in place in shared memory
 #pragma unroll
-      for (int k0 = 0; k0 < kHalfChunks; k0 += kExLdBatch) {
+      for (int k0 = 0; k0 < kExBN / 16; k0 += kExLdBatch) {
         float v[kExLdBatch][16];
         if (ok) {
 #pragma unroll
-          for (int kb = 0; kb < kExLdBatch; ++kb)
-            tmem_ld16(tacc + (half * kHalfChunks + k0 + kb) * 16, v[kb]);
+          for (int kb = 0; kb < kExLdBatch; ++kb) tmem_ld16(tacc + (k0 + kb) * 16, v[kb]);
           tmem_ld_wait();
         }
         if (ok && m < rows) {
 #pragma unroll
           for (int kb = 0; kb < kExLdBatch; ++kb) {
-            const int cc = half * kHalfChunks + k0 + kb;
+            const int cc = k0 + kb;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const int c = 2 * cc + h;
@@ -463,26 +476,21 @@ fused_tc_kernel(const __grid_constant__ FusedTcParams P) {
       }
       tc_fence_before();
       mbar_arrive(tempty0 + 8 * buf);
-      named_bar_sync(1, kExConsumers);
+      named_bar_sync(1 + grp, kFuGroup);  // every row of the tile is updated
+      // (b) coalesced write-back of the rows of the piece: chunk u = j*128 + gt
       const int cend = pe.slices.off[q + 1];
       if (ok) {
-        constexpr int kPer = (kExBM * kExCh) / kExConsumers;
-        uint4 w[kPer];
-#pragma unroll
+        constexpr int kPer = (kExBM * kExCh) / kFuGroup;
+#pragma unroll 4
         for (int j = 0; j < kPer; ++j) {
-          const int u = j * kExConsumers + ct;
-          const int row = u / kExCh, c = u % kExCh;
-          w[j] = *reinterpret_cast<const uint4*>(stage_p + row * (kExBN * 2) +
-                                                 ((c ^ (row & (kExCh - 1))) << 4));
-        }
-#pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-          const int u = j * kExConsumers + ct;
+          const int u = j * kFuGroup + gt;
           const int row = u / kExCh, c = u % kExCh;
           const int col = c0 + 8 * c;
           if (row < rows && col < cend)
             *reinterpret_cast<uint4*>(pe.base + static_cast<int64_t>(trow[row]) * pe.ld_base +
-                                      col) = w[j];
+                                      col) =
+                *reinterpret_cast<const uint4*>(stage_p + row * (kExBN * 2) +
+                                                ((c ^ (row & (kExCh - 1))) << 4));
         }
       }
       mbar_arrive(xempty0 + 8 * s);

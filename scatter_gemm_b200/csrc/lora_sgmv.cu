@@ -519,13 +519,13 @@ lora_status fused_tc(const lora::ShrinkArgs& sa, const lora::ExpandArgs& ea, lor
            static_cast<size_t>(sa.S) * P.rin_bytes +
            static_cast<size_t>(P.base_stages) * lora::kExStageBytes +
            static_cast<size_t>(P.b_stages) * P.btile_bytes + 1024 + 512 +
-           8 * (2 * stages + 1 + 2 * P.b_stages + 4 + 2 * P.base_stages) + 16;
+           8 * (2 * stages + 1 + 2 * P.b_stages + 4 + 2 * 8) + 16;  // <= 8 expand stages
   };
   const int s_min = std::max<int>(2, static_cast<int>((part_bytes + P.stage_bytes - 1) /
                                                       P.stage_bytes));
-  const int rings[3][2] = {{2, LORA_EXPAND_B_STAGES}, {2, 2}, {1, 2}};  // {base, B}
+  const int rings[4][2] = {{2, 6}, {2, LORA_EXPAND_B_STAGES}, {2, 2}, {1, 2}};  // {base, B}
   bool fits = false;
-  for (int i = 0; i < 3 && !fits; ++i) {
+  for (int i = 0; i < 4 && !fits; ++i) {
     P.base_stages = rings[i][0];
     P.b_stages = rings[i][1];
     fits = s_min <= 6 && total(s_min) <= 227 * 1024;
@@ -533,18 +533,21 @@ lora_status fused_tc(const lora::ShrinkArgs& sa, const lora::ExpandArgs& ea, lor
   if (!fits) return LORA_OK;
   P.stages = s_min;
   while (P.stages < 6 && total(P.stages + 1) <= 227 * 1024) ++P.stages;
+  // after the shrink, its ring holds further expand stages (8 in all at most)
+  P.xstages = std::min(8, P.base_stages + static_cast<int>(static_cast<size_t>(P.stages) *
+                                                           P.stage_bytes / lora::kExStageBytes));
   // at least 120 KB, so that two CTAs never share an SM (and its TMEM)
   const size_t smem = std::max<size_t>(total(P.stages), 120 * 1024);
 
-  // cluster size: the largest of 16, 8, 4 CTAs for which every expected piece
-  // (one per 128 rows plus about half a piece per segment) gets a resident
-  // cluster and every CTA at least one K block; otherwise the pair runs unfused
+  // cluster size: the largest of 16, 8, 4 CTAs for which every slot's cluster
+  // (empty ones included: they leave at once, but only after being placed) is
+  // resident at the same time and every CTA has at least one K block;
+  // otherwise the pair runs unfused
   const long slots = lora::num_piece_slots(sa.tok, sa.nseg, lora::kTcBM);
-  const int est = (sa.tok + lora::kTcBM - 1) / lora::kTcBM + (sa.nseg + 1) / 2;
   int cs = 0;
   for (int lg = 4; lg >= 2 && cs == 0; --lg) {
     const int c = 1 << lg;
-    if (c <= dev.max_cluster && P.nkb >= c && est <= dev.fused_clusters[lg]) cs = c;
+    if (c <= dev.max_cluster && P.nkb >= c && slots <= dev.fused_clusters[lg]) cs = c;
   }
   if (cs == 0) return LORA_OK;
   P.csplit = cs;
