@@ -45,6 +45,9 @@ def lib():
             l.oracle_encode_f64.restype = ctypes.c_uint16
             l.oracle_embedding_a.argtypes = [_P, _P, _P, _P, _P, _L] + [_I] * 6
             l.oracle_embedding_a.restype = _I
+            l.oracle_base_expand.argtypes = [_P, _L, _P, _L, _P, _L, _P, _P, _P, _P, _P, _P, _P,
+                                             _L] + [_I] * 9
+            l.oracle_base_expand.restype = _I
             l.oracle_set_threads.argtypes = [_I]
             l.oracle_set_threads.restype = None
             l.oracle_max_threads.argtypes = []
@@ -109,6 +112,21 @@ def embedding_a(ids, A_emb, seg_indptr, weight_indices, out, ld_out, tok, V, r, 
                                     ld_out, tok, V, r, rs, nseg, L)
 
 
+def base_expand(x, ld_x, W, ld_w, in_r, ld_in, B, seg_indptr, weight_indices, permutation,
+                slice_offsets, scalings, out, ld_out, tok, K, S, r, rs, nseg, L, dtype,
+                mode=F32) -> int:
+    """out is modified in place (uint16 for F32, float64 for F64)."""
+    want = np.uint16 if mode == F32 else np.float64
+    assert out.dtype == want and out.flags.c_contiguous
+    x, W, in_r, B = (_c(a, np.uint16) for a in (x, W, in_r, B))
+    si, wi, pm = _c(seg_indptr, np.int32), _c(weight_indices, np.int32), _c(permutation, np.int32)
+    so, sc = _c(slice_offsets, np.int32), _c(scalings, np.float32)
+    return lib().oracle_base_expand(_ptr(x), ld_x, _ptr(W), ld_w, _ptr(in_r), ld_in, _ptr(B),
+                                    _ptr(si), _ptr(wi), _ptr(pm), _ptr(so), _ptr(sc),
+                                    _ptr(out), ld_out, tok, K, S, r, rs, nseg, L, _dt(dtype),
+                                    mode)
+
+
 # ---------------------------------------------------------------- problem helpers
 
 def shrink_problem(p, mode=F32, x=None):
@@ -144,6 +162,24 @@ def expand_problem(p, in_r=None, base=None, mode=F32, scalings=None):
     if rc:
         raise ValueError(f"oracle_expand rejected the problem (code {rc})")
     return out
+
+
+def base_expand_problem(p, W, in_r=None, out=None, mode=F32, scalings=None):
+    """The base projection x W^T with the expand folded in, on a
+    workloads.Problem; W is [N_tot, K] (uint16).  Starts from `out` (default
+    p.base): rows of tokens outside segments keep it."""
+    in_r = p.in_r if in_r is None else in_r
+    sc = p.scalings if scalings is None else scalings
+    if mode == F32:
+        o = (p.base if out is None else out).copy()
+    else:
+        o = np.full(p.base.shape, np.nan, dtype=np.float64)
+    rc = base_expand(p.x, p.ld_x, W, W.shape[1], in_r, in_r.shape[1], p.B, p.seg_indptr,
+                     p.weight_indices, p.permutation, p.slice_offsets, sc, o, p.ld_base,
+                     p.tok, p.K, p.S, p.r, p.rs, p.nseg, p.L, p.dtype, mode)
+    if rc:
+        raise ValueError(f"oracle_base_expand rejected the problem (code {rc})")
+    return o
 
 
 def decode(bits: np.ndarray, dtype: str) -> np.ndarray:

@@ -212,6 +212,71 @@ int oracle_expand(const void* in_r, int64_t ld_in, const uint16_t* B_stack,
 
 /* ---------------------------------------------------------------- embedding A */
 
+/* ---------------------------------------------------------------- base projection + expand
+ *
+ * The expand folded into the base projection that produces its output: on the
+ * sglang page "fused split_qkv / norm / RoPE for Qwen3.5/Next on NPU" (section
+ * of key source snippets, forward_prepare_npu) the qkv_proj output goes
+ * straight to the split step, and with LoRA the expand rewrites that output
+ * first.  The base sum over K and the rank sum over r are kept apart and
+ * combined once, as base + scaling * lora, then rounded. */
+int oracle_base_expand(const uint16_t* x, int64_t ld_x, const uint16_t* W, int64_t ld_w,
+                       const uint16_t* in_r, int64_t ld_in, const uint16_t* B_stack,
+                       const int32_t* seg_indptr, const int32_t* weight_indices,
+                       const int32_t* permutation, const int32_t* slice_offsets,
+                       const float* scalings, void* out, int64_t ld_out, int tok, int K,
+                       int S, int r, int rs, int nseg, int L, int dtype, int mode) {
+  if (K < 1 || r < 1 || rs < r || ld_x < K || ld_w < K || ld_in < (int64_t)S * rs ||
+      (mode != ORACLE_F32 && mode != ORACLE_F64))
+    return ORACLE_BAD_DIMS;
+  int bad = oracle_check_tables(seg_indptr, weight_indices, permutation, slice_offsets,
+                                tok, nseg, L, S, ld_out);
+  if (bad) return bad;
+
+  const int64_t n_tot = (int64_t)slice_offsets[S] - slice_offsets[0];
+
+#pragma omp parallel
+  for (int s = 0; s < nseg; ++s) {
+    const int a = weight_indices[s];
+    const float scaling = scalings[a];
+    const int lo = seg_indptr[s], hi = seg_indptr[s + 1];
+    const uint16_t* B = B_stack + (int64_t)a * n_tot * rs;
+
+#pragma omp for schedule(static) nowait
+    for (int i = lo; i < hi; ++i) {
+      const int64_t t = permutation[i];
+      const uint16_t* xrow = x + t * ld_x;
+      for (int q = 0; q < S; ++q) {
+        const uint16_t* v = in_r + (int64_t)i * ld_in + (int64_t)q * rs;
+        for (int64_t c = slice_offsets[q]; c < slice_offsets[q + 1]; ++c) {
+          const uint16_t* wrow = W + (c - slice_offsets[0]) * ld_w;
+          const uint16_t* brow = B + (c - slice_offsets[0]) * rs;
+          if (mode == ORACLE_F32) {
+            float base = 0.0f;
+            for (int k = 0; k < K; ++k)
+              base += oracle_decode(xrow[k], dtype) * oracle_decode(wrow[k], dtype);
+            float lora = 0.0f;
+            for (int j = 0; j < r; ++j)
+              lora += oracle_decode(v[j], dtype) * oracle_decode(brow[j], dtype);
+            const float sum = scaling == 0.0f ? base : base + scaling * lora;
+            ((uint16_t*)out)[t * ld_out + c] = oracle_encode(sum, dtype);
+          } else {
+            double base = 0.0;
+            for (int k = 0; k < K; ++k)
+              base += (double)oracle_decode(xrow[k], dtype) * (double)oracle_decode(wrow[k], dtype);
+            double lora = 0.0;
+            for (int j = 0; j < r; ++j)
+              lora += (double)oracle_decode(v[j], dtype) * (double)oracle_decode(brow[j], dtype);
+            ((double*)out)[t * ld_out + c] =
+                scaling == 0.0f ? base : base + (double)scaling * lora;
+          }
+        }
+      }
+    }
+  }
+  return 0;
+}
+
 /* The embedding variant of the shrink (sgl-kernel-xpu page, file table:
  * EmbeddingLoraAFwd): the "x" row of a token is the one-hot vector of its id,
  * so the product with A selects one column of the adapter's A. */

@@ -70,6 +70,21 @@ int oracle_expand(const void* in_r, int64_t ld_in, const uint16_t* B_stack,
                   int tok, int S, int r, int rs, int nseg, int L,
                   int dtype, int mode);
 
+/* The base projection with the expand folded into it: for every row i of
+ * segment s (adapter a, token t = permutation[i]) and column c of slice q,
+ *   base = sum_k x[t, k] * W[c - off[0], k]                  (W is [N_tot, ld_w])
+ *   lora = sum_{j<r} in_r[i, q*rs + j] * B[a, c - off[0], j]
+ *   out[t, c] = rn(base + scalings[a] * lora)   (rn(base) when scalings[a] == 0)
+ * with sequential sums (fp32 in ORACLE_F32; fp64 and no rounding in ORACLE_F64,
+ * where out is double).  Only rows of tokens in segments and columns
+ * [off[0], off[S]) are written. */
+int oracle_base_expand(const uint16_t* x, int64_t ld_x, const uint16_t* W, int64_t ld_w,
+                       const uint16_t* in_r, int64_t ld_in, const uint16_t* B_stack,
+                       const int32_t* seg_indptr, const int32_t* weight_indices,
+                       const int32_t* permutation, const int32_t* slice_offsets,
+                       const float* scalings, void* out, int64_t ld_out, int tok, int K,
+                       int S, int r, int rs, int nseg, int L, int dtype, int mode);
+
 /* out[i, j] = A_emb[a, j, ids[i]]  (j < r) for every segment s, a = weight_indices[s],
  * i in [seg_indptr[s], seg_indptr[s+1]); rows are in token order (no permutation).
  * A_emb is [L, rs, V] with the vocabulary dimension contiguous.  Returns

@@ -186,6 +186,20 @@ def _normal_bits(rng, shape, std, dtype):
     return to_bits(rng.standard_normal(shape, dtype=np.float32) * np.float32(std), dtype)
 
 
+def make_base_weight(p: "Problem", seed: int = 0, ld_pad: int = 0) -> np.ndarray:
+    """Seeded base projection weight W [N_tot, K + ld_pad] (uint16 bits) for a
+    problem, output-dimension-major like a linear layer's weight, entries
+    N(0, 1/K) so that x W^T stays of order one; the ld_pad padding columns hold
+    NaN, which no consumer may read."""
+    n_tot = int(p.slice_offsets[-1] - p.slice_offsets[0])
+    rng = np.random.default_rng([seed, 0x57])
+    w = _normal_bits(rng, (n_tot, p.K), 1.0 / np.sqrt(p.K), p.dtype)
+    if ld_pad:
+        w = np.concatenate([w, np.full((n_tot, ld_pad), NAN_BITS[p.dtype], dtype=np.uint16)],
+                           axis=1)
+    return np.ascontiguousarray(w)
+
+
 def make_problem(name: str, seed: int = 0, **over) -> Problem:
     """Builds one seeded instance of workload `name`.
 

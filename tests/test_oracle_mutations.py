@@ -4,7 +4,9 @@ The copy is built in a temporary directory on the CPU; the real oracle is
 never modified.  Every mutation below must make ``test_oracle_pins.py`` fail,
 which shows the pins constrain the gather index, the slice strides of A, B and
 the rank activations, the column offset of B, the scaling, the K range, the
-output row of each op and the orientation of B.
+output row of each op and the orientation of B, and, for the base projection
+with the expand folded in, the column offset of W, its gather row and its
+scaling.
 """
 import os
 import shutil
@@ -38,6 +40,15 @@ MUTATIONS = {
     "expand_row_is_sorted_row": (
         "uint16_t* o = (uint16_t*)base_out + t * ld_base + c;",
         "uint16_t* o = (uint16_t*)base_out + i * ld_base + c;"),
+    "base_W_without_column_offset": (
+        "const uint16_t* wrow = W + (c - slice_offsets[0]) * ld_w;",
+        "const uint16_t* wrow = W + c * ld_w;"),
+    "base_row_is_sorted_row": (
+        "const uint16_t* xrow = x + t * ld_x;",
+        "const uint16_t* xrow = x + (int64_t)i * ld_x;"),
+    "base_scaling_dropped": (
+        "const float sum = scaling == 0.0f ? base : base + scaling * lora;",
+        "const float sum = scaling == 0.0f ? base : base + lora;"),
     "B_transposed": (
         "acc += oracle_decode(v[j], dtype) * oracle_decode(brow[j], dtype);",
         "acc += oracle_decode(v[j], dtype) * "

@@ -14,8 +14,8 @@ import numpy as np
 import pytest
 
 import oracle
-from scatter_gemm_b200.workloads import (CONFIGS, NAN_BITS, from_bits, make_problem,
-                                         to_bits)
+from scatter_gemm_b200.workloads import (CONFIGS, NAN_BITS, from_bits, make_base_weight,
+                                         make_problem, to_bits)
 
 # ----------------------------------------------------------------------------
 # helpers: an independent float64 brute force, token-major
@@ -469,3 +469,68 @@ def test_embedding_a_rejects_out_of_vocabulary_ids():
     out = np.zeros((3, 4), dtype=np.uint16)
     assert oracle.embedding_a(np.array([1, 10, 2]), A, np.array([0, 3]), np.array([0]), out, 4,
                               3, 10, 4, 4, 1, 1) == oracle.BAD_DIMS
+
+
+# ----------------------------------------------------------------------------
+# (f) the base projection with the expand folded in
+# ----------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("seed,dtype", [(40, "bf16"), (41, "fp16"), (42, "bf16")])
+def test_base_expand_matches_token_major_brute_force(seed, dtype):
+    p = tiny_problem(seed, dtype)
+    W = make_base_weight(p, seed, ld_pad=5)
+    Wd = from_bits(W[:, : p.K], dtype).astype(np.float64)
+    X = from_bits(p.x, dtype).astype(np.float64)[:, : p.K]
+    _, delta = dense_reference(p)
+    got = oracle.base_expand_problem(p, W, mode=oracle.F64)
+    off = p.slice_offsets
+    inv = np.empty(p.tok, dtype=np.int64)
+    inv[p.permutation] = np.arange(p.tok)
+    for t in range(p.tok):
+        i = inv[t]
+        in_seg = p.seg_indptr[0] <= i < p.seg_indptr[-1]
+        for c in range(off[0], off[-1]):
+            if in_seg:
+                want = X[t] @ Wd[c - off[0]] + delta[t, c]
+                assert abs(got[t, c] - want) <= 1e-12 * (1 + abs(want))
+            else:
+                assert np.isnan(got[t, c])
+    # nothing outside the slices' columns
+    assert np.isnan(got[:, : off[0]]).all() and np.isnan(got[:, off[-1]:]).all()
+
+
+def test_base_expand_with_zero_weight_is_the_expand_of_zeros():
+    p = tiny_problem(43, "bf16")
+    W = np.zeros((int(p.slice_offsets[-1] - p.slice_offsets[0]), p.K), dtype=np.uint16)
+    zero_base = np.zeros_like(p.base)
+    got = oracle.base_expand_problem(p, W, out=zero_base)
+    want = oracle.expand_problem(p, base=zero_base)
+    assert np.array_equal(got, want)
+
+
+def test_base_expand_with_zero_scaling_is_the_rounded_projection():
+    p = tiny_problem(44, "bf16", K=64)
+    W = make_base_weight(p, 44)
+    z = np.zeros_like(p.scalings)
+    got = from_bits(oracle.base_expand_problem(p, W, scalings=z), "bf16").astype(np.float64)
+    X = from_bits(p.x, "bf16").astype(np.float64)[:, : p.K]
+    Wd = from_bits(W, "bf16").astype(np.float64)
+    off = p.slice_offsets
+    rows = p.permutation[p.seg_indptr[0]: p.seg_indptr[-1]]
+    ref = X[rows] @ Wd.T
+    mag = np.abs(X[rows]) @ np.abs(Wd).T
+    # one rounding to bf16 plus fp32 accumulation over K terms
+    lim = unit_roundoff("bf16") * np.abs(ref) + p.K * 2.0 ** -24 * mag + 1e-30
+    assert (np.abs(got[rows][:, off[0]: off[-1]] - ref) <= lim).all()
+
+
+def test_base_expand_scales_only_the_rank_term():
+    p = tiny_problem(45, "bf16")
+    W = make_base_weight(p, 45)
+    s1 = np.ones_like(p.scalings)
+    base = oracle.base_expand_problem(p, W, mode=oracle.F64, scalings=np.zeros_like(s1))
+    one = oracle.base_expand_problem(p, W, mode=oracle.F64, scalings=s1)
+    three = oracle.base_expand_problem(p, W, mode=oracle.F64, scalings=3 * s1)
+    w = ~np.isnan(base)
+    np.testing.assert_allclose((three - base)[w], 3 * (one - base)[w], rtol=1e-12, atol=1e-12)
