@@ -210,6 +210,52 @@ def time_fused(probs, lora, flush, stream, steps, warmup, nap):
     return out
 
 
+def time_base_expand(lora, flush, stream, device, toks, steps, warmup, nap):
+    """lora_base_expand (the projection with the expand folded in) on the qkv
+    workload, beside the unfused route: cuBLAS x W^T (torch.matmul) then
+    lora_expand.  Timed like the sweep (L2 flushed, GPU sleep, CUDA events);
+    reported beside `value`, which the pages' two ops define."""
+    out = []
+    for tok in toks:
+        p = W.make_problem("qkv", seed=7, tok=tok)
+        dp = DevProblem(p, device)
+        tdt = dp.x.dtype
+        wt = torch.from_numpy(W.make_base_weight(p, 7).view(np.int16)).to(device).view(tdt)
+        inr = torch.from_numpy(p.in_r.view(np.int16)).to(device).view(tdt)
+        res = dp.base.clone()
+        xk = dp.x[:, : p.K]
+
+        def fused():
+            lora.lora_base_expand(xk, wt, inr, dp.B, dp.si, dp.wi, dp.pm, dp.off, dp.sc, res,
+                                  rank=p.r)
+
+        def separate():
+            torch.matmul(xk, wt.t(), out=res[:, dp.off[0]: dp.off[-1]])
+            lora.lora_expand(inr, dp.B, dp.si, dp.wi, dp.pm, dp.off, dp.sc, res, rank=p.r,
+                             workspace=dp.ws)
+
+        ms = {}
+        for name, fn in (("fused", fused), ("separate", separate)):
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(steps)]
+            for k in range(warmup + steps):
+                flush.zero_()
+                torch.cuda._sleep(nap)
+                if k >= warmup:
+                    ev[k - warmup][0].record(stream)
+                fn()
+                if k >= warmup:
+                    ev[k - warmup][1].record(stream)
+            torch.cuda.synchronize()
+            ms[name] = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+        flops = 2.0 * tok * (dp.off[-1] - dp.off[0]) * p.K + 2.0 * tok * (dp.off[-1] - dp.off[0]) * p.r
+        tf = flops / (ms["fused"] * 1e-3) / 1e12
+        out.append({"tok": tok, "fused_us": round(ms["fused"] * 1e3, 1),
+                    "cublas_plus_expand_us": round(ms["separate"] * 1e3, 1),
+                    "tflops": round(tf, 1)})
+    return out
+
+
 # ----------------------------------------------------------------------------
 # CPU oracle timing (baseline; never the product path)
 # ----------------------------------------------------------------------------
@@ -342,6 +388,10 @@ def run_ours(args, rank, world, device):
     fused = None
     if not args.no_fused:
         fused = time_fused(probs, lora, flush, stream, min(args.steps, 200), 3, nap)
+    base_fused = None
+    if not args.no_base_expand:
+        base_fused = time_base_expand(lora, flush, stream, device, (512, 2048, 8192),
+                                      min(args.steps, 20), 3, nap)
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, probs, lora, device, stream, world)
@@ -419,6 +469,7 @@ def run_ours(args, rank, world, device):
         "mean_case_gbs": round(mean_case, 1),
         "per_tok": detail,
         "fused_decode": fused,
+        "base_expand": base_fused,
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -486,6 +537,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-fused", action="store_true")
+    ap.add_argument("--no-base-expand", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

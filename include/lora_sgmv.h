@@ -276,6 +276,32 @@ LORA_API lora_status lora_shrink_expand(const void* x, int64_t ld_x, const void*
                                         int nseg, int L, lora_dtype dtype, void* workspace,
                                         size_t workspace_bytes, void* stream);
 
+/* lora_base_expand -- the base projection with the expand folded into it.
+ *   out[perm[i], c] = rn( sum_k x[perm[i], k] * W[c - off[0], k]
+ *                         + scalings[a] * sum_{j<r} in_r[i, q*rs + j] * B_stack[a, c - off[0], j] )
+ * for the rows i of every segment (adapter a) and the columns c of slice q;
+ * rn(projection) alone where scalings[a] == 0.  On the sglang page for
+ * Qwen3.5/Next on NPU (key source snippets, forward_prepare_npu) the qkv_proj
+ * output goes straight to the split step: computing it with the LoRA term
+ * included writes it once, instead of writing it and then reading and
+ * rewriting it in lora_expand.
+ *   x [tok, ld_x], W [N_tot, ld_w] (the projection weight, output-dimension-
+ *   major, K contiguous), in_r [tok, ld_in] (sorted order, as lora_expand),
+ *   B_stack [L, N_tot, rs], slice_offsets (HOST, S+1), scalings [L] fp32,
+ *   out [tok, ld_out >= off[S]]: written at the rows of tokens in segments and
+ *   columns [off[0], off[S]); nothing else.
+ * The two sums are formed in fp32 (the projection over K on the tensor cores)
+ * and rounded once.  Tensor-core layout only: x, W, in_r, B_stack, out 16-byte
+ * aligned, K, rs, ld_* and slice starts multiples of 8, r <= 64; otherwise
+ * LORA_ERR_UNSUPPORTED.  Other errors as lora_expand. */
+LORA_API lora_status lora_base_expand(const void* x, int64_t ld_x, const void* W, int64_t ld_w,
+                                      const void* in_r, int64_t ld_in, const void* B_stack,
+                                      const int32_t* seg_indptr, const int32_t* weight_indices,
+                                      const int32_t* permutation, const int32_t* slice_offsets,
+                                      const float* scalings, void* out, int64_t ld_out,
+                                      int tok, int K, int S, int r, int rs, int nseg, int L,
+                                      lora_dtype dtype, void* stream);
+
 /* ---- 64-bit index tables ------------------------------------------------
  * lora_shrink_i64 / lora_expand_i64 take seg_indptr, weight_indices and
  * permutation as int64_t (the default index type of PyTorch), as the

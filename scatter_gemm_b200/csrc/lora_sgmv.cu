@@ -24,6 +24,7 @@
 #include "common.cuh"
 #include "embedding.cuh"
 #include "expand_tc.cuh"
+#include "base_expand_tc.cuh"
 #include "fused_tc.cuh"
 #include "general.cuh"
 #include "group.cuh"
@@ -97,6 +98,8 @@ void set_kernel_attrs() {
                        cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   cudaFuncSetAttribute(lora::fused_tc_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        227 * 1024);
+  cudaFuncSetAttribute(lora::base_expand_tc_kernel<E>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   cudaFuncSetAttribute(lora::fused_tc_kernel<E>, cudaFuncAttributeNonPortableClusterSizeAllowed,
                        1);
 }
@@ -995,4 +998,118 @@ extern "C" lora_status lora_shrink_expand(
                                      stream);
   g_last_path |= path;
   return s2;
+}
+
+// ------------------------------------------------------------------ base projection + expand
+
+namespace {
+
+template <class E>
+lora_status base_expand_tc(const lora::BaseExpandArgs& a, const void* W, int64_t ld_w,
+                           const void* B_stack, lora_dtype dt, cudaStream_t st) {
+  lora::BaseExpandTcParams P;
+  std::memset(&P, 0, sizeof(P));
+  P.a = a;
+  P.rpad = a.r <= 16 ? 16 : (a.r <= 32 ? 32 : 64);
+  P.sw_layout = P.rpad == 16 ? 6u : (P.rpad == 32 ? 4u : 2u);
+  const CUtensorMapSwizzle swz = P.rpad == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                 : P.rpad == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                : CU_TENSOR_MAP_SWIZZLE_128B;
+  P.rin_bytes = lora::kTcBM * P.rpad * 2;
+  P.btile_bytes = lora::kBeBN * P.rpad * 2;
+  P.idesc = lora::make_idesc_f16(dt == LORA_BF16 ? 1 : 0, lora::kTcBM, lora::kBeBN);
+  P.nkb = (a.K + lora::kTcAtomK - 1) / lora::kTcAtomK;
+  int tiles = 0;
+  for (int q = 0; q < a.S; ++q) {
+    P.tile_prefix[q] = tiles;
+    tiles += (a.slices.off[q + 1] - a.slices.off[q] + lora::kBeBN - 1) / lora::kBeBN;
+  }
+  for (int q = a.S; q <= LORA_MAX_SLICES; ++q) P.tile_prefix[q] = tiles;
+  if (tiles == 0) return LORA_OK;
+  P.tiles_total = tiles;
+
+  // K ring of 32 KB stages; two CTAs per SM when three stages fit in 113 KB
+  constexpr size_t kStage = lora::kTcBM * 128 + lora::kBeBN * 128;
+  auto total = [&](int stages) {
+    return static_cast<size_t>(stages) * kStage + P.rin_bytes + P.btile_bytes + 1024 + 512 +
+           8 * (2 * stages + 3) + 16;
+  };
+  const bool two = total(3) <= 113 * 1024;
+  const size_t cap = (two ? 113 : 225) * 1024;
+  P.stages = 2;
+  while (P.stages < 6 && total(P.stages + 1) <= cap) ++P.stages;
+  if (total(P.stages) > 225 * 1024) return LORA_ERR_UNSUPPORTED;
+  // at least 80 KB: never more than two CTAs (2 x 256 TMEM columns) on an SM
+  const size_t smem = std::max<size_t>(total(P.stages), 80 * 1024);
+
+  const int64_t n_tot = a.slices.off[a.S] - a.slices.off[0];
+  if (!encode_2d(&P.tmap_W, dt, W, a.K, static_cast<uint64_t>(n_tot),
+                 static_cast<uint64_t>(ld_w) * 2, lora::kTcAtomK, lora::kBeBN,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&P.tmap_B, dt, B_stack, a.r, static_cast<uint64_t>(a.L) * n_tot,
+                 static_cast<uint64_t>(a.rs) * 2, P.rpad, lora::kBeBN, swz))
+    return LORA_ERR_CUDA;
+
+  const long slots = lora::num_piece_slots(a.tok, a.nseg, lora::kTcBM);
+  if (slots * tiles >= (1L << 31)) return LORA_ERR_UNSUPPORTED;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(slots * tiles));
+  cfg.blockDim = dim3(lora::kBeThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, lora::base_expand_tc_kernel<E>, P);
+  ++g_launches;
+  g_last_path = LORA_PATH_TENSOR | LORA_PATH_FUSED;
+  return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" lora_status lora_base_expand(
+    const void* x, int64_t ld_x, const void* W, int64_t ld_w, const void* in_r, int64_t ld_in,
+    const void* B_stack, const int32_t* seg_indptr, const int32_t* weight_indices,
+    const int32_t* permutation, const int32_t* slice_offsets, const float* scalings, void* out,
+    int64_t ld_out, int tok, int K, int S, int r, int rs, int nseg, int L, lora_dtype dtype,
+    void* stream) {
+  if (dtype != LORA_BF16 && dtype != LORA_FP16) return LORA_ERR_UNSUPPORTED;
+  if (tok < 0 || nseg < 0 || K < 1 || S < 1 || r < 1 || rs < r || L < 1)
+    return LORA_ERR_INVALID_ARGUMENT;
+  if (S > LORA_MAX_SLICES) return LORA_ERR_UNSUPPORTED;
+  if (!slice_offsets) return LORA_ERR_INVALID_ARGUMENT;
+  if (ld_x < K || ld_w < K || ld_in < static_cast<int64_t>(S) * rs)
+    return LORA_ERR_INVALID_ARGUMENT;
+  lora::SliceTable tab{};
+  tab.S = S;
+  for (int q = 0; q <= S; ++q) {
+    tab.off[q] = slice_offsets[q];
+    if (slice_offsets[q] < 0 || slice_offsets[q] > ld_out) return LORA_ERR_INVALID_ARGUMENT;
+    if (q > 0 && slice_offsets[q] < slice_offsets[q - 1]) return LORA_ERR_INVALID_ARGUMENT;
+  }
+  if (tok == 0 || nseg == 0 || tab.off[S] == tab.off[0]) return LORA_OK;
+  if (!x || !W || !in_r || !B_stack || !seg_indptr || !weight_indices || !scalings || !out)
+    return LORA_ERR_INVALID_ARGUMENT;
+  if (!aligned_to(seg_indptr, 4) || !aligned_to(weight_indices, 4) ||
+      !aligned_to(scalings, 4) || (permutation && !aligned_to(permutation, 4)))
+    return LORA_ERR_INVALID_ARGUMENT;
+  // tensor-core layout: 16-byte rows and slice starts (no element-aligned path)
+  if (!aligned_to(x, 16) || !aligned_to(W, 16) || !aligned_to(in_r, 16) ||
+      !aligned_to(B_stack, 16) || !aligned_to(out, 16) || (ld_x % 8) || (ld_w % 8) ||
+      (ld_in % 8) || (ld_out % 8) || (K % 8) || (rs % 8) || r > 64)
+    return LORA_ERR_UNSUPPORTED;
+  for (int q = 0; q <= S; ++q)
+    if (tab.off[q] % 8) return LORA_ERR_UNSUPPORTED;
+  const int64_t n_tot = tab.off[S] - tab.off[0];
+  if (static_cast<int64_t>(L) * n_tot >= (int64_t(1) << 31) || tok >= (1 << 30))
+    return LORA_ERR_UNSUPPORTED;
+
+  const lora::BaseExpandArgs a{static_cast<const uint16_t*>(x), ld_x,
+                               static_cast<const uint16_t*>(in_r), ld_in, seg_indptr,
+                               weight_indices, permutation, scalings,
+                               static_cast<uint16_t*>(out), ld_out, tok, K, S, r, rs, nseg, L,
+                               tab};
+  const DeviceFacts* dev = device_facts();
+  if (!dev) return LORA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return dtype == LORA_BF16 ? base_expand_tc<lora::Bf16>(a, W, ld_w, B_stack, dtype, st)
+                            : base_expand_tc<lora::Fp16>(a, W, ld_w, B_stack, dtype, st);
 }

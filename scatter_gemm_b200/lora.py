@@ -74,6 +74,9 @@ def lib() -> ctypes.CDLL:
             l.lora_shrink_expand.argtypes = [_P, _L, _P, _P, _P, _P, _P, _P, _P, _P, _L, _P, _L] + \
                 [_I] * 8 + [_P, _Z, _P]
             l.lora_shrink_expand.restype = _I
+            l.lora_base_expand.argtypes = [_P, _L, _P, _L, _P, _L, _P, _P, _P, _P, _P, _P, _P,
+                                           _L] + [_I] * 8 + [_P]
+            l.lora_base_expand.restype = _I
             _lib = l
     return _lib
 
@@ -340,6 +343,53 @@ def lora_shrink_expand(x: torch.Tensor, A_stack: torch.Tensor, B_stack: torch.Te
     if st != LORA_OK:
         raise LoraError("lora_shrink_expand", st)
     return base_out
+
+
+def lora_base_expand(x: torch.Tensor, W: torch.Tensor, in_r: torch.Tensor,
+                     B_stack: torch.Tensor, seg_indptr: torch.Tensor,
+                     weight_indices: torch.Tensor, permutation: Optional[torch.Tensor],
+                     slice_offsets: Sequence[int], scalings: torch.Tensor, out: torch.Tensor, *,
+                     rank: Optional[int] = None, stream=None) -> torch.Tensor:
+    """The base projection with the expand folded in:
+    out[perm[i], c] = rn(x[perm[i]] . W[c-off0] + s_a * in_r[i, q*rs:q*rs+r] . B_a[c-off0, :r])
+    for the rows of every segment and the columns of the slices.
+
+    x [tok, K], W [N_tot, >= K] (unit inner stride), in_r [tok, >= S*rs],
+    B_stack [L, N_tot, rs], out [tok, >= off[S]] (written there only)."""
+    dt = _dtype_code(x)
+    for t, n in ((W, "W"), (in_r, "in_r"), (B_stack, "B_stack"), (out, "out")):
+        if t.dtype != x.dtype:
+            raise TypeError(f"{n} must have the element type of x")
+    if scalings.dtype != torch.float32 or not scalings.is_cuda or not scalings.is_contiguous():
+        raise ValueError("scalings must be a contiguous fp32 CUDA tensor")
+    ld_x = _row_major(x, "x")
+    ld_w = _row_major(W, "W")
+    ld_in = _row_major(in_r, "in_r")
+    ld_out = _row_major(out, "out")
+    if B_stack.dim() != 3 or not B_stack.is_contiguous():
+        raise ValueError("B_stack must be a contiguous [L, N_tot, rs] tensor")
+    L, n_tot, rs = B_stack.shape
+    off = [int(v) for v in (slice_offsets.tolist() if torch.is_tensor(slice_offsets)
+                            else slice_offsets)]
+    S = len(off) - 1
+    if S < 1 or S > MAX_SLICES or off[-1] - off[0] != n_tot or W.shape[0] != n_tot:
+        raise ValueError("slice_offsets, W and B_stack disagree on N_tot")
+    tok, K = x.shape
+    if W.shape[1] < K or in_r.shape[0] != tok or out.shape[0] != tok:
+        raise ValueError("x, W, in_r and out disagree on tok or K")
+    r = rs if rank is None else int(rank)
+    nseg = seg_indptr.numel() - 1
+    off_arr = (ctypes.c_int32 * len(off))(*off)
+    st = lib().lora_base_expand(x.data_ptr(), ld_x, W.data_ptr(), ld_w, in_r.data_ptr(), ld_in,
+                                B_stack.data_ptr(), _table(seg_indptr, "seg_indptr"),
+                                _table(weight_indices, "weight_indices"),
+                                _table(permutation, "permutation", True),
+                                ctypes.cast(off_arr, ctypes.c_void_p), scalings.data_ptr(),
+                                out.data_ptr(), ld_out, tok, K, S, r, rs, nseg, L, dt,
+                                _stream(stream))
+    if st != LORA_OK:
+        raise LoraError("lora_base_expand", st)
+    return out
 
 
 def lora_validate(seg_indptr: torch.Tensor, weight_indices: torch.Tensor,

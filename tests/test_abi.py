@@ -176,6 +176,32 @@ def test_shrink_expand_argument_checks(L, kw, want):
     assert pair(L, **kw) == want
 
 
+def base_expand(lib, off=(0, 32, 40, 48), **kw):
+    arr = (ctypes.c_int32 * len(off))(*off)
+    a = dict(x=P, ld_x=64, W=P, ld_w=64, inr=P, ld_in=48, B=P, si=P, wi=P, pm=P,
+             offp=ctypes.cast(arr, ctypes.c_void_p), sc=P, out=P, ld_out=48, tok=10, K=64,
+             S=len(off) - 1, r=16, rs=16, nseg=2, nad=4, dt=0, st=None)
+    a.update(kw)
+    return lib.lora_base_expand(a["x"], a["ld_x"], a["W"], a["ld_w"], a["inr"], a["ld_in"],
+                                a["B"], a["si"], a["wi"], a["pm"], a["offp"], a["sc"], a["out"],
+                                a["ld_out"], a["tok"], a["K"], a["S"], a["r"], a["rs"],
+                                a["nseg"], a["nad"], a["dt"], a["st"])
+
+
+# all of these return before any CUDA call
+@pytest.mark.parametrize("kw,want", [
+    (dict(x=None), INVALID), (dict(W=None), INVALID), (dict(inr=None), INVALID),
+    (dict(B=None), INVALID), (dict(sc=None), INVALID), (dict(out=None), INVALID),
+    (dict(offp=None), INVALID), (dict(ld_w=32), INVALID), (dict(ld_in=40), INVALID),
+    (dict(ld_out=40), INVALID), (dict(K=0), INVALID), (dict(dt=2), UNSUPPORTED),
+    (dict(x=P + 2), UNSUPPORTED), (dict(W=P + 8), UNSUPPORTED), (dict(ld_w=68), UNSUPPORTED),
+    (dict(K=60, ld_x=64, ld_w=64), UNSUPPORTED), (dict(r=65, rs=72, ld_in=3 * 72), UNSUPPORTED),
+    (dict(pm=P + 2), INVALID), (dict(tok=0), OK), (dict(nseg=0), OK),
+])
+def test_base_expand_argument_checks(L, kw, want):
+    assert base_expand(L, **kw) == want
+
+
 def test_index64_workspace_size(L):
     # narrowed seg_indptr, weight_indices and permutation, each padded to 16 bytes
     assert lora.index64_workspace_size(100, 3) == 4 * (4 + 4 + 100)
