@@ -250,14 +250,14 @@ int oracle_base_expand(const uint16_t* x, int64_t ld_x, const uint16_t* W, int64
         const uint16_t* v = in_r + (int64_t)i * ld_in + (int64_t)q * rs;
         for (int64_t c = slice_offsets[q]; c < slice_offsets[q + 1]; ++c) {
           const uint16_t* wrow = W + (c - slice_offsets[0]) * ld_w;
-          const uint16_t* brow = B + (c - slice_offsets[0]) * rs;
+          const uint16_t* bcol = B + (c - slice_offsets[0]) * rs;  /* B row of column c */
           if (mode == ORACLE_F32) {
             float base = 0.0f;
             for (int k = 0; k < K; ++k)
               base += oracle_decode(xrow[k], dtype) * oracle_decode(wrow[k], dtype);
             float lora = 0.0f;
             for (int j = 0; j < r; ++j)
-              lora += oracle_decode(v[j], dtype) * oracle_decode(brow[j], dtype);
+              lora += oracle_decode(v[j], dtype) * oracle_decode(bcol[j], dtype);
             const float sum = scaling == 0.0f ? base : base + scaling * lora;
             ((uint16_t*)out)[t * ld_out + c] = oracle_encode(sum, dtype);
           } else {
@@ -266,7 +266,7 @@ int oracle_base_expand(const uint16_t* x, int64_t ld_x, const uint16_t* W, int64
               base += (double)oracle_decode(xrow[k], dtype) * (double)oracle_decode(wrow[k], dtype);
             double lora = 0.0;
             for (int j = 0; j < r; ++j)
-              lora += (double)oracle_decode(v[j], dtype) * (double)oracle_decode(brow[j], dtype);
+              lora += (double)oracle_decode(v[j], dtype) * (double)oracle_decode(bcol[j], dtype);
             ((double*)out)[t * ld_out + c] =
                 scaling == 0.0f ? base : base + (double)scaling * lora;
           }
