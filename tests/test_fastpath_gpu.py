@@ -84,6 +84,17 @@ def test_expand_tile_runs_per_cta(tok):
     assert lora.last_path() & T
 
 
+# Segments that start off the 128-row grid add partial pieces; aligned ones
+# leave the segment-start slots empty.  Both layouts, at sizes where several
+# CTAs share each piece's column tiles.
+@pytest.mark.parametrize("tok,recipe", [(2048, "dirichlet"), (6144, "dirichlet"),
+                                        (6144, "uniform")])
+def test_expand_aligned_and_ragged_segment_layouts(tok, recipe):
+    p = make_problem("qkv", seed=30, tok=tok, K=64, nseg=8, L=8, recipe=recipe)
+    check_expand(p)
+    assert lora.last_path() & T
+
+
 def test_expand_empty_slice_and_single_column_tiles():
     p = make_problem("qkv", seed=28, tok=200, K=64, slices=[128, 0, 8, 120, 0, 136])
     check_expand(p)
