@@ -89,10 +89,10 @@ enum {
   LORA_PATH_FUSED = 16   /* lora_shrink_expand ran both ops in one launch            */
 };
 
-/* Limits of this build. */
+/* Compile-time limits of the library. */
 #define LORA_MAX_SLICES 8
 
-/* lora_shrink -- the shrink of the chunked-SGMV pair (page section "Summary").
+/* lora_shrink -- the shrink of the chunked-SGMV pair (sgl-kernel-xpu page, section "Summary").
  *
  *   out_r[i, q*rs + j] = round( sum_{k<K} x[permutation[i], k] * A_stack[a, q*rs + j, k] )
  *   for every segment s, a = weight_indices[s], i in its rows, q < S, j < r.
@@ -116,7 +116,7 @@ LORA_API lora_status lora_shrink(const void* x, int64_t ld_x, const void* A_stac
                         lora_dtype dtype, void* workspace, size_t workspace_bytes,
                         void* stream);
 
-/* lora_expand -- the expand of the chunked-SGMV pair (page section "Summary").
+/* lora_expand -- the expand of the chunked-SGMV pair (sgl-kernel-xpu page, section "Summary").
  *
  *   for every segment s with a = weight_indices[s] and scalings[a] != 0, every row i of s,
  *   every slice q < S and column c in [slice_offsets[q], slice_offsets[q+1]):
@@ -147,7 +147,7 @@ LORA_API lora_status lora_expand(const void* in_r, int64_t ld_in, const void* B_
  * adapter-grouped schedule for tables with many small segments. */
 LORA_API size_t lora_workspace_size(int tok, int nseg, int L);
 
-/* lora_validate -- the value checks of the tables (page section "Behaviour
+/* lora_validate -- the value checks of the tables (sgl-kernel-xpu page, section "Behaviour
  * changes": seg_indptr, index range, permutation, offset table), run on the
  * device.  Writes the OR of the LORA_BAD_* bits that apply into *d_result
  * (device int32, overwritten; 0 = valid).  slice_offsets is a HOST array and
