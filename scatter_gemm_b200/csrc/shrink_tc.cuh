@@ -211,12 +211,16 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
         mbar_arrive(full0 + 8 * ((i - lag) % P.stages));
       }
     }
-    // drain: publish the stages still in flight
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
+    // drain: publish the stages still in flight, oldest first, each as soon
+    // as this thread's copies of it have landed
     if (ok) {
-      for (int i = max(0, nk - lag); i < nk; ++i) mbar_arrive(full0 + 8 * (i % P.stages));
+      for (int i = max(0, nk - lag); i < nk; ++i) {
+        cp_async_wait_dyn(nk - 1 - i);
+        fence_proxy_async_smem();
+        mbar_arrive(full0 + 8 * (i % P.stages));
+      }
     }
+    cp_async_wait<0>();
   } else if (warp == 4) {
     // =========================== MMA issuer
     if (lane == 0) {
@@ -323,7 +327,9 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
         if (ok && n < nvalid && (n % p.rs) < p.r) orow[n] = E::f32_to_bits(sv[k]);
       }
     }
-    cluster_sync();  // peers are done reading this CTA's partial
+    // peers are done reading this CTA's partial (their loads have returned:
+    // the sums above used them), so the arrive needs no release ordering
+    cluster_sync_relaxed();
   }
 
   __syncthreads();

@@ -271,6 +271,15 @@ __device__ __forceinline__ void cluster_sync() {
                    : "memory");
 }
 
+// Cluster barrier whose arrive carries no release ordering.  For a kernel's
+// last barrier, which only keeps this CTA's shared memory alive until every
+// peer has finished reading it: a peer's remote loads are complete once their
+// values have been used, and its global stores need not be acknowledged first.
+__device__ __forceinline__ void cluster_sync_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" :::
+                   "memory");
+}
+
 __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
