@@ -168,6 +168,7 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
     constexpr int RSTEP = kTcBM / CPR;            // rows between a thread's chunks
     const int cc = tid % CPR;                     // this thread's chunk column
     const int rr = tid / CPR;                     // ... and first row
+    const int wrow0 = (tid & ~31) / CPR;          // first row of this warp
     const uint32_t sub_off = (cc >> 3) * (kTcBM * 128);  // x sub-tile of this chunk
     const uint32_t a_sub = P.npad * 128;  // one 64-K sub-tile of A
     const uint32_t a_bytes = kTcNSub * a_sub;
@@ -192,16 +193,29 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
       }
       const int k = k0 + 8 * cc;
       const bool k_in = k < p.K;
-#pragma unroll
-      for (int j = 0; j < CPR; ++j) {
-        // every row is copied, zero-filled past the piece and past K: a
-        // predicated copy keeps this issue loop (the shrink's bottleneck)
-        // free of branches, which measured faster than skipping those rows
+      // Row j of this thread: zero-filled past the piece and past K, so the
+      // copies of a warp never diverge.
+      auto copy_row = [&](int j) {
         const int row = rr + j * RSTEP;
         const bool in = k_in && row < rows;
         const uint32_t dst = xs + sub_off + row * 128 + (((cc & 7) ^ (row & 7)) << 4);
         cp_async_16(dst, in ? static_cast<const void*>(xr[j] + k) : static_cast<const void*>(p.x),
                     in ? 16u : 0u);
+      };
+      if (rows >= kTcBM) {
+#pragma unroll
+        for (int j = 0; j < CPR; ++j) copy_row(j);
+      } else {
+        // A short piece: a warp stops once its first row for this j is past
+        // the piece (warp-uniform, and true for every later j).  Those stage
+        // rows are not written; the accumulator rows they feed are never
+        // stored or reduced.  (Full pieces keep the loop without the test,
+        // which measured faster for them.)
+#pragma unroll
+        for (int j = 0; j < CPR; ++j) {
+          if (wrow0 + j * RSTEP >= rows) break;
+          copy_row(j);
+        }
       }
       cp_async_commit();
       if (i >= lag) {
