@@ -11,10 +11,6 @@
 //   expand; otherwise the element-aligned CUDA-core kernels of general.cuh.
 //   With a workspace and more segments than adapters the tensor-core kernels
 //   run on the adapter-grouped schedule of group.cuh.
-// The other entry points: lora_shrink_expand (fused_tc for decode-sized
-// batches, else the pair), lora_base_expand (base_expand_tc), the int64-table
-// forms (narrow_index_kernel, then the pair), the fixed-slice and embedding
-// forms, and lora_validate.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
