@@ -232,12 +232,16 @@ LORA_API lora_status lora_embedding_a(const int32_t* ids, const void* A_emb,
  * (1 MiB) compiled into the library, which every GPU that loads the library
  * holds until the process exits.
  *
- *  - Limit: lora_workspace_size(tok, nseg, L) must not exceed
+ *  - Limit: only calls with more segments than adapters (nseg > L) use the
+ *    scratch.  For them lora_workspace_size(tok, nseg, L) must not exceed
  *    LORA_STATIC_SCRATCH_BYTES (about tok + nseg + L <= 262,000); larger
- *    problems return LORA_ERR_UNSUPPORTED before anything is enqueued.
+ *    problems return LORA_ERR_UNSUPPORTED before anything is enqueued.  Calls
+ *    with nseg <= L need no scratch and have no such limit.
  *  - The first call on each device looks up the array's device address with
  *    that device current (a CUDA runtime query, no allocation) and caches it;
- *    make that first call before any stream capture.
+ *    make that first call before any stream capture.  The cached address
+ *    belongs to the device's context at that time: resetting the device
+ *    (cudaDeviceReset) after the first call is not supported.
  *  - Every call on a device shares the one array and leaves its contents
  *    behind; nothing in it has to start at zero.  Calls whose kernels overlap
  *    on the GPU (e.g. on two streams) race on the array: serialise them.

@@ -862,6 +862,11 @@ extern "C" lora_status lora_shrink_static_scratch(
     const void* x, int64_t ld_x, const void* A_stack, const int32_t* seg_indptr,
     const int32_t* weight_indices, const int32_t* permutation, void* out_r, int64_t ld_out,
     int tok, int K, int S, int r, int rs, int nseg, int L, lora_dtype dtype, void* stream) {
+  // Only the adapter-grouping pass uses scratch, and it runs only with more
+  // segments than adapters; any other call needs none, so it has no size limit.
+  if (!(nseg > L && L <= lora::kGroupMaxAdapters))
+    return lora_shrink(x, ld_x, A_stack, seg_indptr, weight_indices, permutation, out_r,
+                       ld_out, tok, K, S, r, rs, nseg, L, dtype, nullptr, 0, stream);
   // the grouping pass writes every word of the scratch it later reads, so
   // nothing has to be cleared between calls
   if (lora_workspace_size(tok, nseg, L) > LORA_STATIC_SCRATCH_BYTES) return LORA_ERR_UNSUPPORTED;

@@ -184,17 +184,10 @@ def _ws(workspace: Optional[torch.Tensor]):
     return workspace.data_ptr(), workspace.numel() * workspace.element_size()
 
 
-def lora_shrink(x: torch.Tensor, A_stack: torch.Tensor, seg_indptr: torch.Tensor,
-                weight_indices: torch.Tensor, permutation: Optional[torch.Tensor],
-                out_r: torch.Tensor, *, num_slices: int, rank: Optional[int] = None,
-                workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """Shrink: out_r[i, q*rs+j] = sum_k x[perm[i], k] * A_stack[a, q*rs+j, k].
-
-    x [tok, K] (unit inner stride), A_stack [L, S*rs, K] contiguous (or
-    [L, S, rs, K]), out_r [tok, >= S*rs] (unit inner stride, sorted order).
-    `rank` is the valid rank r <= rs (default rs).  The index tables are all
-    int32, or all int64 (then lora_shrink_i64 runs, and a workspace is
-    allocated when none is given)."""
+def _shrink_shapes(x: torch.Tensor, A_stack: torch.Tensor, out_r: torch.Tensor,
+                   num_slices: int, rank: Optional[int]):
+    """Host-side shape checks shared by the shrink entry points; returns
+    (dtype code, ld_x, ld_out, tok, K, S, r, rs, L)."""
     dt = _dtype_code(x)
     if A_stack.dtype != x.dtype or out_r.dtype != x.dtype:
         raise TypeError("x, A_stack and out_r must share one element type")
@@ -203,6 +196,8 @@ def lora_shrink(x: torch.Tensor, A_stack: torch.Tensor, seg_indptr: torch.Tensor
     if not A_stack.is_contiguous():
         raise ValueError("A_stack must be contiguous")
     S = int(num_slices)
+    if S < 1:
+        raise ValueError("num_slices must be positive")
     if A_stack.dim() == 4:
         L, S4, rs, K = A_stack.shape
         if S4 != S:
@@ -220,6 +215,23 @@ def lora_shrink(x: torch.Tensor, A_stack: torch.Tensor, seg_indptr: torch.Tensor
     r = rs if rank is None else int(rank)
     if out_r.shape[0] != tok:
         raise ValueError("out_r must have one row per token")
+    if out_r.shape[1] < S * rs:
+        raise ValueError(f"out_r must have at least S*rs = {S * rs} columns")
+    return dt, ld_x, ld_out, tok, K, S, r, rs, L
+
+
+def lora_shrink(x: torch.Tensor, A_stack: torch.Tensor, seg_indptr: torch.Tensor,
+                weight_indices: torch.Tensor, permutation: Optional[torch.Tensor],
+                out_r: torch.Tensor, *, num_slices: int, rank: Optional[int] = None,
+                workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Shrink: out_r[i, q*rs+j] = sum_k x[perm[i], k] * A_stack[a, q*rs+j, k].
+
+    x [tok, K] (unit inner stride), A_stack [L, S*rs, K] contiguous (or
+    [L, S, rs, K]), out_r [tok, >= S*rs] (unit inner stride, sorted order).
+    `rank` is the valid rank r <= rs (default rs).  The index tables are all
+    int32, or all int64 (then lora_shrink_i64 runs, and a workspace is
+    allocated when none is given)."""
+    dt, ld_x, ld_out, tok, K, S, r, rs, L = _shrink_shapes(x, A_stack, out_r, num_slices, rank)
     nseg = seg_indptr.numel() - 1
     idt = _index_dtype(seg_indptr, weight_indices, permutation)
     if idt == torch.int64:
@@ -433,25 +445,14 @@ def lora_shrink_static_scratch(x: torch.Tensor, A_stack: torch.Tensor, seg_indpt
     library's own fixed 1 MiB device array holds the scratch.  Calls that
     overlap on the GPU race on that array, and problems whose workspace would
     exceed it raise LoraError (LORA_ERR_UNSUPPORTED)."""
-    l = lib()
-    f = l.lora_shrink_static_scratch
+    dt, ld_x, ld_out, tok, K, S, r, rs, L = _shrink_shapes(x, A_stack, out_r, num_slices, rank)
+    f = lib().lora_shrink_static_scratch
     f.argtypes = [_P, _L, _P, _P, _P, _P, _P, _L] + [_I] * 8 + [_P]
     f.restype = _I
-    dt = _dtype_code(x)
-    if A_stack.dtype != x.dtype or out_r.dtype != x.dtype:
-        raise TypeError("x, A_stack and out_r must share one element type")
-    if A_stack.dim() != 3 or not A_stack.is_contiguous():
-        raise ValueError("A_stack must be a contiguous [L, S*rs, K] tensor")
-    S = int(num_slices)
-    L, srs, K = A_stack.shape
-    rs = srs // S
-    r = rs if rank is None else int(rank)
-    tok = x.shape[0]
-    st = f(x.data_ptr(), _row_major(x, "x"), A_stack.data_ptr(),
+    st = f(x.data_ptr(), ld_x, A_stack.data_ptr(),
            _table(seg_indptr, "seg_indptr"), _table(weight_indices, "weight_indices"),
-           _table(permutation, "permutation", True), out_r.data_ptr(),
-           _row_major(out_r, "out_r"), tok, K, S, r, rs, seg_indptr.numel() - 1, L, dt,
-           _stream(stream))
+           _table(permutation, "permutation", True), out_r.data_ptr(), ld_out,
+           tok, K, S, r, rs, seg_indptr.numel() - 1, L, dt, _stream(stream))
     if st != LORA_OK:
         raise LoraError("lora_shrink_static_scratch", st)
     return out_r

@@ -231,3 +231,28 @@ def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(lora, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         lora.lib()
+
+
+@pytest.mark.parametrize("fn", ["lora_shrink", "lora_shrink_static_scratch"])
+@pytest.mark.parametrize("case", ["short_out", "narrow_out", "narrow_x", "ragged_slices"])
+def test_shrink_bindings_check_shapes_before_any_call(L, fn, case):
+    """Both shrink bindings reject mismatched shapes on the host, before the
+    library is called (the tensors here are CPU tensors: nothing reaches a GPU)."""
+    import torch
+    tok, K, S, rs = 12, 64, 3, 16
+    x = torch.zeros(tok, K, dtype=torch.bfloat16)
+    A = torch.zeros(2, S * rs, K, dtype=torch.bfloat16)
+    out = torch.zeros(tok, S * rs, dtype=torch.bfloat16)
+    S_arg = S
+    if case == "short_out":
+        out = torch.zeros(tok - 1, S * rs, dtype=torch.bfloat16)
+    elif case == "narrow_out":
+        out = torch.zeros(tok, S * rs - 8, dtype=torch.bfloat16)
+    elif case == "narrow_x":
+        x = torch.zeros(tok, 2 * K, dtype=torch.bfloat16)[:, : K - 8]
+    else:
+        S_arg = 5  # 48 rows of A are not a multiple of 5 slices
+    si = torch.zeros(2, dtype=torch.int32)
+    wi = torch.zeros(1, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        getattr(lora, fn)(x, A, si, wi, None, out, num_slices=S_arg)

@@ -3,10 +3,11 @@
 Some callers are handed only input and output buffers by a host framework and
 cannot allocate device memory, so they cannot pass the workspace that the
 adapter-grouped schedule needs.  This entry point keeps that scratch in a
-fixed array inside the library.  Its results must match the ordinary
-lora_shrink called with a caller-provided workspace, call after call, and it
-must refuse problems whose scratch would not fit.  The file is named to be
-collected last.
+fixed array inside the library.  Its results must match the CPU oracle and the
+ordinary lora_shrink called with a caller-provided workspace, call after call;
+it must refuse problems whose scratch would not fit, and calls that need no
+scratch (no more segments than adapters) must have no size limit.  The file is
+named to be collected last.
 """
 import ctypes
 
@@ -14,6 +15,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from scatter_gemm_b200 import lora
 from scatter_gemm_b200.workloads import make_problem
 from tests.devutil import SENTINEL, Guarded, assert_close, tables
@@ -41,6 +43,10 @@ def test_static_scratch_shrink_matches_the_workspace_shrink_twice():
     assert lora.last_path() & lora.PATH_GROUPED
     ref_bits = ref.bits()
     written = ref_bits != SENTINEL
+    # the oracle (its sentinel marks the rows and columns it leaves unwritten)
+    want = oracle.shrink_problem(p)
+    want_written = want != 0x7FFF
+    assert np.array_equal(written, want_written), "write set differs from the oracle's"
 
     for call in range(2):
         out = Guarded(np.full((p.tok, p.S * p.rs), SENTINEL, np.uint16), dt)
@@ -60,6 +66,7 @@ def test_static_scratch_shrink_matches_the_workspace_shrink_twice():
         assert out.guards_intact()
         assert np.array_equal(got[~written], ref_bits[~written]), f"call {call}: write set"
         assert_close(got[written], ref_bits[written], p.dtype, what=f"call {call}")
+        assert_close(got[written], want[written], p.dtype, what=f"call {call} vs oracle")
     assert lora.device_error(clear=True) == 0
 
 
@@ -91,3 +98,23 @@ def test_static_scratch_refuses_problems_beyond_its_size():
     P = 0x10000  # never dereferenced: the size check comes first
     st = f(P, 64, P, P, P, P, P, 48, too_many, 64, 3, 16, 16, 1024, 64, 0, None)
     assert st == lora.LORA_ERR_UNSUPPORTED
+
+
+def test_static_scratch_without_grouping_has_no_size_limit():
+    # no more segments than adapters: the call needs no scratch, so a token
+    # count whose grouping workspace would exceed the array still runs
+    tok, K, S, rs, L = 270_000, 64, 1, 8, 4
+    assert lora.workspace_size(tok, L, L) > lora.STATIC_SCRATCH_BYTES
+    g = torch.Generator(device="cuda").manual_seed(5)
+    x = torch.randn(tok, K, device="cuda", generator=g).to(torch.bfloat16)
+    A = (0.02 * torch.randn(L, S * rs, K, device="cuda", generator=g)).to(torch.bfloat16)
+    si = torch.tensor([0, 60_000, 130_000, 200_000, tok], dtype=torch.int32, device="cuda")
+    wi = torch.tensor([2, 0, 3, 1], dtype=torch.int32, device="cuda")
+    pm = torch.randperm(tok, device="cuda", generator=g).to(torch.int32)
+    ref = torch.zeros(tok, S * rs, dtype=torch.bfloat16, device="cuda")
+    lora.lora_shrink(x, A, si, wi, pm, ref, num_slices=S)
+    got = torch.zeros_like(ref)
+    lora.lora_shrink_static_scratch(x, A, si, wi, pm, got, num_slices=S)
+    torch.cuda.synchronize()
+    assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+    assert lora.device_error(clear=True) == 0
