@@ -147,11 +147,16 @@ class DevProblem:
     def __init__(self, p, device):
         self.p = p
         tdt = torch.bfloat16 if p.dtype == "bf16" else torch.float16
+        mis = int(p.misalign)  # elements past a 16-byte boundary (the tail workload: 2)
 
         def up(bits):
-            return torch.from_numpy(bits.view(np.int16)).to(device).view(tdt)
+            # every data tensor starts `mis` elements into its allocation
+            flat = torch.from_numpy(np.ascontiguousarray(bits).reshape(-1).view(np.int16))
+            buf = torch.zeros(flat.numel() + mis + 8, dtype=torch.int16, device=device)
+            buf[mis: mis + flat.numel()].copy_(flat)
+            return buf[mis: mis + flat.numel()].view(tdt).view(*bits.shape)
 
-        self.x = up(p.x)
+        self.x = up(p.x)[:, : p.K]
         self.A = up(p.A)
         self.B = up(p.B)
         self.base = up(p.base)
@@ -159,7 +164,7 @@ class DevProblem:
         self.wi = torch.from_numpy(p.weight_indices).to(device)
         self.pm = torch.from_numpy(p.permutation).to(device)
         self.sc = torch.from_numpy(p.scalings).to(device)
-        self.out = torch.zeros(p.tok, p.S * p.rs, dtype=tdt, device=device)
+        self.out = up(np.zeros((p.tok, p.S * p.rs), dtype=np.uint16))
         self.off = [int(v) for v in p.slice_offsets]
         from scatter_gemm_b200 import lora
         self.ws = lora.make_workspace(p.tok, p.nseg, p.L, device)
@@ -256,9 +261,105 @@ def time_base_expand(lora, flush, stream, device, toks, steps, warmup, nap):
     return out
 
 
+# the other workloads of the pages' "Performance"/"Testing" sections, one line
+# each (the headline `value` stays the qkv sweep)
+CONFIG_LINES = (("tiny", "bf16"), ("gate_up", "bf16"), ("gate_up", "fp16"), ("tail", "fp16"),
+                ("many_small", "bf16"))
+
+
+def path_names(bits, lora):
+    names = [("tensor", lora.PATH_TENSOR), ("general", lora.PATH_GENERAL),
+             ("grouped", lora.PATH_GROUPED), ("splitk", lora.PATH_SPLITK),
+             ("fused", lora.PATH_FUSED)]
+    return "+".join(n for n, b in names if bits & b)
+
+
+def time_configs(lora, flush, stream, device, steps, warmup, nap, peak, which=CONFIG_LINES):
+    """Shrink and expand of each workload in `which`, timed like the sweep (L2
+    flushed and a GPU sleep before each call, CUDA events around it)."""
+    out = []
+    for name, dt in which:
+        p = W.make_problem(name, seed=0, dtype=dt)
+        dp = DevProblem(p, device)
+        row = {"config": name, "dtype": dt, "tok": p.tok, "K": p.K,
+               "slices": [int(v) for v in np.diff(p.slice_offsets)], "rank": p.r,
+               "adapters": p.L, "segments": p.nseg, "misalign_elems": p.misalign}
+        for op, fn, nbytes in (("shrink", dp.shrink, dp.bytes_shrink),
+                               ("expand", dp.expand, dp.bytes_expand)):
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(steps)]
+            for k in range(warmup + steps):
+                flush.zero_()
+                torch.cuda._sleep(nap)
+                if k >= warmup:
+                    ev[k - warmup][0].record(stream)
+                fn(lora)
+                if k >= warmup:
+                    ev[k - warmup][1].record(stream)
+            torch.cuda.synchronize()
+            t = [a.elapsed_time(b) for a, b in ev]
+            ms = float(np.mean(t))
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            row[f"{op}_us"] = round(ms * 1e3, 2)
+            row[f"{op}_us_median"] = round(float(np.median(t)) * 1e3, 2)
+            row[f"{op}_mb"] = round(nbytes / 1e6, 2)
+            row[f"{op}_gbs"] = round(gbs, 1)
+            row[f"{op}_frac_of_measured"] = round(gbs / peak, 4)
+            row[f"{op}_frac_of_nominal_8tbs"] = round(gbs / NOMINAL_HBM_GBS, 4)
+            row[f"{op}_path"] = path_names(lora.last_path(), lora)
+        out.append(row)
+        del dp
+    return out
+
+
 # ----------------------------------------------------------------------------
 # CPU oracle timing (baseline; never the product path)
 # ----------------------------------------------------------------------------
+
+# bounded samples of each workload for the per-config CPU baseline: the
+# workload's own recipe at a smaller token count where the full one would take
+# the oracle more than a few seconds on one thread
+CPU_SAMPLES = (("tiny", "bf16", {}), ("qkv", "bf16", {"tok": 512}),
+               ("gate_up", "bf16", {"tok": 128}), ("gate_up", "fp16", {"tok": 128}),
+               ("tail", "fp16", {}), ("many_small", "bf16", {"tok": 256, "nseg": 32}))
+
+
+def time_oracle_configs(reps=3):
+    """The oracle on one thread and on all host threads, median of `reps`
+    runs of shrink + expand, per workload sample (GB/s of algorithmic bytes)."""
+    import oracle
+    all_threads = oracle.max_threads()
+    rows = []
+    for name, dt, over in CPU_SAMPLES:
+        p = W.make_problem(name, seed=0, dtype=dt, **over)
+        nbytes = W.bytes_shrink(p) + W.bytes_expand(p)
+        row = {"config": name, "dtype": dt, "tok": p.tok, "segments": p.nseg,
+               "mb": round(nbytes / 1e6, 2)}
+        for label, n in (("single", 1), ("all", all_threads)):
+            oracle.set_threads(n)
+            ts = []
+            for _ in range(reps):
+                t0 = time.perf_counter()
+                h = oracle.shrink_problem(p)
+                oracle.expand_problem(p, in_r=h)
+                ts.append(time.perf_counter() - t0)
+            row[f"{label}_s"] = round(statistics.median(ts), 4)
+            row[f"{label}_gbs"] = round(nbytes / statistics.median(ts) / 1e9, 4)
+        rows.append(row)
+    oracle.set_threads(all_threads)
+    return rows, all_threads
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
 
 def time_oracle(toks, min_seconds):
     import oracle
@@ -278,37 +379,49 @@ def time_oracle(toks, min_seconds):
 
 
 def run_reference(args, rank, world):
-    """--impl reference: the CPU oracle timed on the host cores, rank 0 only."""
+    """--impl reference: the CPU oracle timed on the host cores, rank 0 only,
+    on the same nine-token sweep as our arm: a step is shrink + expand at every
+    tok of the sweep (about 1.5 s of oracle work on the host's threads).  With
+    more than 60 timed steps a step covers one tok of the sweep, in rotation,
+    so that the run stays within minutes; the bytes and times still add up over
+    the sweep."""
     if rank != 0:
         return
     import oracle
-    toks = (50,)
+    toks = [int(t) for t in args.toks.split(",")]
     probs = [W.make_problem("qkv", seed=0, tok=t) for t in toks]
-    nbytes = sum(W.bytes_shrink(p) + W.bytes_expand(p) for p in probs)
+    full = args.steps <= 60
 
-    def step():
-        for p in probs:
+    def step_problems(k):
+        return probs if full else [probs[k % len(probs)]]
+
+    for k in range(min(args.warmup, 1)):
+        for p in step_problems(k):
             h = oracle.shrink_problem(p)
             oracle.expand_problem(p, in_r=h)
-
-    for _ in range(args.warmup):
-        step()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
-    el = time.perf_counter() - t0
-    value = nbytes * args.steps / el / 1e9
+    nbytes = 0
+    el = 0.0
+    for k in range(args.steps):
+        for p in step_problems(k):
+            nbytes += W.bytes_shrink(p) + W.bytes_expand(p)
+            t0 = time.perf_counter()
+            h = oracle.shrink_problem(p)
+            oracle.expand_problem(p, in_r=h)
+            el += time.perf_counter() - t0
+    value = nbytes / el / 1e9
     cores = oracle.max_threads()
-    sample = ("one shrink + expand of the tok=50 case of the sweep per step "
+    sample = ("shrink + expand at every tok of the sweep per step (CPU oracle, fp32 sequential "
+              "sums, OpenMP over the rows of a segment)" if full else
+              "shrink + expand at one tok of the sweep per step, in rotation over the sweep "
               "(CPU oracle, fp32 sequential sums)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample": sample},
+        "config": {"workload": WORKLOAD, "toks": toks, "sample": sample},
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -392,6 +505,13 @@ def run_ours(args, rank, world, device):
     if not args.no_base_expand:
         base_fused = time_base_expand(lora, flush, stream, device, (512, 2048, 8192),
                                       min(args.steps, 20), 3, nap)
+    configs = None
+    if not args.no_configs:
+        which = CONFIG_LINES
+        if args.configs:
+            which = tuple(tuple(c.split(":")) for c in args.configs.split(","))
+        configs = time_configs(lora, flush, stream, device, min(args.steps, 100), 3, nap,
+                               measured_peaks()[0], which)
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, probs, lora, device, stream, world)
@@ -448,7 +568,13 @@ def run_ours(args, rank, world, device):
         v, el, passes, cores = time_oracle([50, 128, 256, 512, 1024], args.cpu_seconds)
         cpu = {"value": round(v, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
                "sample": f"tok 50,128,256,512,1024 of the sweep, shrink + expand, "
-                         f"{passes} pass(es) in {el:.1f} s"}
+                         f"{passes} pass(es) in {el:.1f} s, all host threads",
+               "nproc": os.cpu_count(), "cpu_model": cpu_model()}
+        if not args.no_configs:
+            rows, _ = time_oracle_configs()
+            cpu["per_config"] = rows
+            cpu["per_config_note"] = ("median of 3 runs of shrink + expand on one thread and "
+                                      "on all host threads, per workload sample")
 
     value = bytes_step * args.steps * world / (kernel_ms * 1e-3) / 1e9
     line = {
@@ -468,6 +594,7 @@ def run_ours(args, rank, world, device):
         "geomean_frac_nominal_tok_ge_1024": round(geo / NOMINAL_HBM_GBS, 4) if geo else None,
         "mean_case_gbs": round(mean_case, 1),
         "per_tok": detail,
+        "per_config": configs,
         "fused_decode": fused,
         "base_expand": base_fused,
         "roofline": roof,
@@ -538,6 +665,9 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-fused", action="store_true")
     ap.add_argument("--no-base-expand", action="store_true")
+    ap.add_argument("--no-configs", action="store_true")
+    ap.add_argument("--configs", default="",
+                    help="per-config lines to time, e.g. gate_up:fp16,tail:fp16 (default: all)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -37,7 +37,20 @@
  *  - Nothing is synchronised with the host: the calls read no table on the
  *    host, enqueue their kernels on `stream` (a cudaStream_t, NULL = legacy
  *    default stream) and return.  The library allocates no device memory and
- *    keeps no state between calls; calls are thread-safe.
+ *    keeps no state between calls; calls may be made from several host
+ *    threads and on several streams at once.  Kernels of calls that overlap on
+ *    the GPU never wait for each other: every kernel that holds tensor memory
+ *    (TMEM) takes at most 256 of an SM's 512 columns and enough shared memory
+ *    that at most two of its thread blocks share an SM.  The exception is other
+ *    software's kernels: a kernel outside this library that holds more TMEM
+ *    on an SM while it waits for thread blocks elsewhere can make a thread
+ *    block of this library wait for its TMEM; do not overlap such kernels with
+ *    these calls.
+ *  - Every wait of a kernel on an mbarrier gives up after 1 s, records an
+ *    error code (lora_device_error) and lets the kernel finish without
+ *    writing further results.  Thread-block-cluster barriers and the TMEM
+ *    allocation are not bounded this way; the rule above keeps them from
+ *    waiting on anything but the cluster's own thread blocks.
  *  - Invalid table VALUES (a decreasing seg_indptr, an adapter index out of
  *    range, a permutation that is not a bijection) are undefined behaviour in
  *    lora_shrink / lora_expand, as on the pages (section "Behaviour changes");

@@ -131,13 +131,17 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * P.b_stages + 5 +
                                                     2 * P.base_stages);
 
-  // Barriers (one consumer thread) and TMEM (warp 0) first, in different warps,
-  // so that both overlap the table reads.
-  if (tid == 32) {
+  // Barriers (one consumer thread; the B ring's by warp 0, which uses them
+  // before the CTA barrier) and TMEM (warp 0) first, so that both overlap the
+  // table reads.
+  if (tid == 0) {
     for (int s = 0; s < P.b_stages; ++s) {
       mbar_init(bfull0 + 8 * s, 1);
       mbar_init(bempty0 + 8 * s, 1);
     }
+    fence_mbar_init();
+  }
+  if (tid == 32) {
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull0 + 8 * b, 1);
       mbar_init(tempty0 + 8 * b, kExConsumers);
@@ -217,6 +221,18 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
     }
   };
   const int pre = min(P.base_stages, ntl);  // tiles issued before the CTA barrier
+  // The first B tiles depend only on the adapter: warp 0 requests them now,
+  // before the row tokens are known and the CTA barrier is passed.
+  const int pre_b = min(P.b_stages, ntl);
+  if (tid == 0) {
+    for (int t = 0; t < pre_b; ++t) {
+      int q, c0;
+      tile_info(t, q, c0);
+      mbar_arrive_expect_tx(bfull0 + 8 * t, P.btile_bytes);
+      tma_load_2d(bring + t * P.btile_bytes, &P.tmap_B, bfull0 + 8 * t, 0,
+                  static_cast<int>(adapter * n_tot + (c0 - off0)));
+    }
+  }
 
   if (producer) {
     // Row tables, then every load that needs no barrier goes out before the
@@ -265,14 +281,6 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
   if (warp == 0) {
     // =========================== B tiles (TMA) and MMA issue
     if (lane == 0) {
-      const int pre = min(P.b_stages, ntl);
-      for (int t = 0; t < pre; ++t) {
-        int q, c0;
-        tile_info(t, q, c0);
-        mbar_arrive_expect_tx(bfull0 + 8 * t, P.btile_bytes);
-        tma_load_2d(bring + t * P.btile_bytes, &P.tmap_B, bfull0 + 8 * t, 0,
-                    static_cast<int>(adapter * n_tot + (c0 - off0)));
-      }
       ok = mbar_wait(rin_bar, 0);
       for (int t = 0; t < ntl && ok; ++t) {
         const int s = t % P.b_stages, buf = t & 1;

@@ -22,9 +22,10 @@
 // requested while the shrink runs.
 //
 // Roles (416 threads):
-//   warp 0      TMEM (512 columns: shrink accumulator at column 0, the expand's
-//               double-buffered accumulator at column 256); A and B tiles by
-//               TMA; every MMA;
+//   warp 0      TMEM (256 columns: first the shrink accumulator, then, once it
+//               has been read out and the cluster has passed its barriers, the
+//               expand's double-buffered accumulator); A and B tiles by TMA;
+//               every MMA;
 //   warps 1-8   expand epilogue as two groups of four warps taking alternate
 //               tiles (group g uses accumulator buffer g); warps 1-4 also read
 //               the shrink accumulator out into the split-K partial;
@@ -42,8 +43,8 @@
 namespace lora {
 
 constexpr int kFuThreads = 416;
-constexpr int kFuTmemCols = 512;
-constexpr int kFuExpandCol = 256;  // first TMEM column of the expand accumulators
+constexpr int kFuTmemCols = 256;
+constexpr int kFuExpandCol = 0;    // the expand accumulators reuse the shrink's columns
 constexpr int kFuGroup = 128;      // threads of one consumer group (four warps)
 
 struct FusedTcParams {

@@ -153,6 +153,12 @@ expand_general_kernel(const ExpandArgs p) {
   const int q = slice_of(p.slices, c);
   const int64_t n_tot = p.slices.off[p.S] - off0;
   const uint16_t* brow = p.B + ((int64_t)a * n_tot + (c - off0)) * p.rs;
+  // the base elements of this column first: their loads stay in flight while
+  // the rank sums are formed
+  uint16_t old[kGBM];
+#pragma unroll
+  for (int m = 0; m < kGBM; ++m)
+    old[m] = m < rows ? p.base[(int64_t)tok_of_row[m] * p.ld_base + c] : uint16_t(0);
 
   float acc[kGBM];
 #pragma unroll
@@ -171,12 +177,10 @@ expand_general_kernel(const ExpandArgs p) {
     }
   }
 #pragma unroll
-  for (int m = 0; m < kGBM; ++m) {
-    if (m >= rows) break;
-    uint16_t* o = p.base + (int64_t)tok_of_row[m] * p.ld_base + c;
-    const float out = E::bits_to_f32(*o) + scale * acc[m];
-    *o = E::f32_to_bits(out);
-  }
+  for (int m = 0; m < kGBM; ++m)
+    if (m < rows)
+      p.base[(int64_t)tok_of_row[m] * p.ld_base + c] =
+          E::f32_to_bits(E::bits_to_f32(old[m]) + scale * acc[m]);
 }
 
 // ---------------------------------------------------------------------------

@@ -24,6 +24,7 @@
 #include "common.cuh"
 #include "embedding.cuh"
 #include "expand_tc.cuh"
+#include "expand_unaligned_tc.cuh"
 #include "base_expand_tc.cuh"
 #include "fused_tc.cuh"
 #include "general.cuh"
@@ -48,6 +49,9 @@
 #ifndef LORA_EXPAND_B_STAGES
 #define LORA_EXPAND_B_STAGES 3
 #endif
+#ifndef LORA_SHRINK_WIDE_SMEM
+#define LORA_SHRINK_WIDE_SMEM 0     // 1: one-CTA-per-SM budget when the grid fits the SMs
+#endif
 
 namespace {
 
@@ -55,6 +59,14 @@ thread_local uint64_t g_launches = 0;
 thread_local int g_last_path = 0;
 
 constexpr int kMaxDevices = 64;
+
+// Every kernel of this library that holds TMEM allocates at most 256 columns
+// and asks for at least this much dynamic shared memory, so that no more than
+// two of its CTAs fit on one SM (228 KB) and their allocations (2 x 256 of 512
+// columns) never wait for each other, whatever calls run concurrently on
+// other streams: a CTA blocked in tcgen05.alloc while its cluster peers hold
+// TMEM and wait at a cluster barrier could otherwise deadlock.
+constexpr size_t kTmemCtaMinSmem = 80 * 1024;
 
 inline bool aligned_to(const void* p, uintptr_t a) {
   return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
@@ -79,23 +91,26 @@ struct DeviceFacts {
 DeviceFacts g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
-template <class E, int NSUB>
+template <class E, int NSUB, bool AL>
 void set_shrink_attrs() {
-  cudaFuncSetAttribute(lora::shrink_tc_kernel<E, NSUB>,
+  cudaFuncSetAttribute(lora::shrink_tc_kernel<E, NSUB, AL>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-  cudaFuncSetAttribute(lora::shrink_tc_kernel<E, NSUB>,
+  cudaFuncSetAttribute(lora::shrink_tc_kernel<E, NSUB, AL>,
                        cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
 }
 
 template <class E>
 void set_kernel_attrs() {
-  set_shrink_attrs<E, 1>();
-  set_shrink_attrs<E, 2>();
-  set_shrink_attrs<E, 4>();
+  set_shrink_attrs<E, 1, true>();
+  set_shrink_attrs<E, 2, true>();
+  set_shrink_attrs<E, 4, true>();
+  set_shrink_attrs<E, 1, false>();
   cudaFuncSetAttribute(lora::expand_tc_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        227 * 1024);
   cudaFuncSetAttribute(lora::expand_general_kernel<E>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  cudaFuncSetAttribute(lora::expand_unaligned_kernel<E>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   cudaFuncSetAttribute(lora::fused_tc_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        227 * 1024);
   cudaFuncSetAttribute(lora::base_expand_tc_kernel<E>,
@@ -130,7 +145,7 @@ const DeviceFacts* device_facts() {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int nclusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&nclusters, lora::shrink_tc_kernel<lora::Bf16, 1>,
+    if (cudaOccupancyMaxActiveClusters(&nclusters, lora::shrink_tc_kernel<lora::Bf16, 1, true>,
                                        &cfg) ==
             cudaSuccess &&
         nclusters > 0)
@@ -299,11 +314,16 @@ lora_status shrink_general(const lora::ShrinkArgs& a, cudaStream_t st) {
   return launch_status();
 }
 
+// The tensor-core shrink: aligned (16-byte rows, TMA for A) or element-aligned
+// (row staging and shifts); the CUDA-core kernel only beyond 256 outputs.
 bool shrink_tc_eligible(const lora::ShrinkArgs& a) {
   const int npad = round_up(a.S * a.rs, 16);
-  return aligned_to(a.x, 16) && (a.ld_x % 8) == 0 && (a.K % 8) == 0 && aligned_to(a.A, 16) &&
-         npad <= 256 && static_cast<int64_t>(a.L) * a.S * a.rs < (int64_t(1) << 31) &&
+  return npad <= 256 && static_cast<int64_t>(a.L) * a.S * a.rs < (int64_t(1) << 31) &&
          a.tok < (1 << 30);
+}
+
+bool shrink_tc_aligned(const lora::ShrinkArgs& a) {
+  return aligned_to(a.x, 16) && (a.ld_x % 8) == 0 && (a.K % 8) == 0 && aligned_to(a.A, 16);
 }
 
 template <class E>
@@ -317,40 +337,73 @@ lora_status shrink_tc(const lora::ShrinkArgs& a, lora_dtype dt, const Grouping& 
   P.nvseg = g.vseg_indptr ? g.nvseg : a.nseg;
   P.npad = round_up(a.S * a.rs, 16);
   P.tmem_cols = P.npad <= 32 ? 32 : P.npad <= 64 ? 64 : P.npad <= 128 ? 128 : 256;
-  // widest stage (64-K sub-tiles of x and A) that still leaves two stages, and
-  // room for the split-K partial, inside the shared-memory budget
-  const int budget = (LORA_SHRINK_CTAS_PER_SM >= 2 && P.npad <= 128 ? 110 : 220) * 1024;
-  const size_t part_bytes = sizeof(float) * lora::kTcBM * (P.npad + 4);
-  int nsub = lora::kTcMaxNSub;
+  // widest stage (64-K sub-tiles of x and A) that still leaves two stages
+  // inside the shared-memory budget
+  int budget = (LORA_SHRINK_CTAS_PER_SM >= 2 && P.npad <= 128 ? 110 : 220) * 1024;
+  const bool al = shrink_tc_aligned(a);
+  int nsub = al ? lora::kTcMaxNSub : 1;
   for (;; nsub /= 2) {
     const int sb = nsub * (lora::kTcBM * 128 + P.npad * 128);
-    if (nsub == 1 || (2 * sb <= budget - 2048 && static_cast<size_t>(2 * sb) >= part_bytes)) break;
+    if (nsub == 1 || 2 * sb <= budget - 2048) break;
   }
   P.stage_bytes = nsub * (lora::kTcBM * 128 + P.npad * 128);
-  P.stages = (budget - 2048) / static_cast<int>(P.stage_bytes);
-  P.stages = P.stages < 2 ? 2 : (P.stages > 8 ? 8 : P.stages);
-  while (static_cast<size_t>(P.stages) * P.stage_bytes < part_bytes) ++P.stages;
+  if (!al)  // plus the staging of x rows and A rows
+    P.stage_bytes = static_cast<uint32_t>(round_up(
+        static_cast<int>(P.stage_bytes) + (lora::kTcBM + P.npad) * lora::kRawRow, 1024));
   P.nkb = (a.K + nsub * lora::kTcAtomK - 1) / (nsub * lora::kTcAtomK);
 
+  if (al && !encode_2d(&P.tmap_A, dt, a.A, a.K, static_cast<uint64_t>(a.L) * a.S * a.rs,
+                       static_cast<uint64_t>(a.K) * 2, lora::kTcAtomK, P.npad,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+    return LORA_ERR_CUDA;
   // K split over a cluster: the smallest power of two that gives every SM a CTA
   // (expected pieces: one per 128 rows plus about half a piece per segment),
   // keeping at least four stages of K per CTA.  (Splitting further, to fill
   // every resident CTA slot, measured slower: more partials to reduce.)
-  if (!encode_2d(&P.tmap_A, dt, a.A, a.K, static_cast<uint64_t>(a.L) * a.S * a.rs,
-                 static_cast<uint64_t>(a.K) * 2, lora::kTcAtomK, P.npad,
-                 CU_TENSOR_MAP_SWIZZLE_128B))
-    return LORA_ERR_CUDA;
-  const size_t smem_need = static_cast<size_t>(P.stages) * P.stage_bytes + 1024 +
-                           8 * (2 * P.stages + 2) + 8 * lora::kTcBM + 16;
   const int est = (a.tok + lora::kTcBM - 1) / lora::kTcBM + (P.vseg_indptr ? a.L : a.nseg) / 2;
+  // a grid that fits one CTA per SM may use the shared memory of two, with
+  // clusters of at most 8 (two per GPC at one CTA per SM)
+  const long nslots = lora::num_piece_slots(a.tok, P.nvseg, lora::kTcBM);
+  const bool wide = LORA_SHRINK_WIDE_SMEM && nslots * 8 <= dev.sms;
+  const int max_cs = wide ? std::min(dev.max_cluster, 8) : dev.max_cluster;
   int cs = 1;
-  while (cs < dev.max_cluster && P.nkb >= 4 * cs &&
-         (est * cs < dev.sms || cs < LORA_SHRINK_MIN_SPLIT))
+  while (cs < max_cs && P.nkb >= 4 * cs && (est * cs < dev.sms || cs < LORA_SHRINK_MIN_SPLIT))
     cs *= 2;
+#ifdef LORA_SHRINK_FORCE_CS
+  cs = LORA_SHRINK_FORCE_CS;
+  if (P.nkb < cs) cs = 1;
+#endif
   P.csplit = cs;
   P.kb_per = (P.nkb + cs - 1) / cs;
   P.idesc = lora::make_idesc_f16(dt == LORA_BF16 ? 1 : 0, lora::kTcBM, P.npad);
-
+  P.vec_out = aligned_to(a.out, 16) && (a.ld_out % 8) == 0;
+  // ring stages in what the split-K receive buffer leaves of the budget; when
+  // the whole grid fits one CTA per SM, the budget of one CTA per SM
+  if (wide && nslots * cs <= dev.sms) budget = 220 * 1024;
+#ifdef LORA_SHRINK_FORCE_WIDE
+  budget = LORA_SHRINK_FORCE_WIDE ? 220 * 1024 : 110 * 1024;
+#endif
+  const size_t recv_full = cs > 1 ? static_cast<size_t>(lora::kTcBM) * P.npad * 4 : 0;
+  auto smem_for = [&](int stages, size_t recv) {
+    return static_cast<size_t>(stages) * P.stage_bytes + recv + 1024 + 8 * (2 * stages + 3) +
+           8 * lora::kTcBM;
+  };
+  auto stages_for = [&](size_t recv) {
+    int st = 2;
+    while (st < 8 && smem_for(st + 1, recv) <= static_cast<size_t>(budget)) ++st;
+    return st;
+  };
+  // a separate receive buffer when it leaves at least three stages; otherwise
+  // the partials are received in the ring after a cluster barrier
+  P.stages = stages_for(recv_full);
+  P.recv_in_ring = 0;
+  if (cs > 1 && P.stages < 3) {
+    P.recv_in_ring = 1;
+    P.stages = stages_for(0);
+    while (static_cast<size_t>(P.stages) * P.stage_bytes < recv_full) ++P.stages;
+  }
+  const size_t smem_need =
+      std::max<size_t>(smem_for(P.stages, P.recv_in_ring ? 0 : recv_full), kTmemCtaMinSmem);
   const size_t smem = smem_need;
   const long slots = lora::num_piece_slots(a.tok, P.nvseg, lora::kTcBM);
   cudaLaunchConfig_t cfg{};
@@ -369,9 +422,10 @@ lora_status shrink_tc(const lora::ShrinkArgs& a, lora_dtype dt, const Grouping& 
   }
   if (smem > 227 * 1024) return LORA_ERR_UNSUPPORTED;
   cudaError_t e;
-  if (nsub == 4) e = cudaLaunchKernelEx(&cfg, lora::shrink_tc_kernel<E, 4>, P);
-  else if (nsub == 2) e = cudaLaunchKernelEx(&cfg, lora::shrink_tc_kernel<E, 2>, P);
-  else e = cudaLaunchKernelEx(&cfg, lora::shrink_tc_kernel<E, 1>, P);
+  if (!al) e = cudaLaunchKernelEx(&cfg, lora::shrink_tc_kernel<E, 1, false>, P);
+  else if (nsub == 4) e = cudaLaunchKernelEx(&cfg, lora::shrink_tc_kernel<E, 4, true>, P);
+  else if (nsub == 2) e = cudaLaunchKernelEx(&cfg, lora::shrink_tc_kernel<E, 2, true>, P);
+  else e = cudaLaunchKernelEx(&cfg, lora::shrink_tc_kernel<E, 1, true>, P);
   ++g_launches;
   g_last_path = LORA_PATH_TENSOR | (cs > 1 ? LORA_PATH_SPLITK : 0) |
                 (P.vseg_indptr ? LORA_PATH_GROUPED : 0);
@@ -448,7 +502,7 @@ lora_status expand_tc(const lora::ExpandArgs& a, lora_dtype dt, const Grouping& 
   if (total(P.base_stages) > 225 * 1024) return LORA_ERR_UNSUPPORTED;
   size_t smem = total(P.base_stages);
   // keep the CTAs per SM within TMEM: 512 columns / kExTmemCols
-  const size_t min_smem = lora::kExTmemCols > 256 ? 116 * 1024 : 80 * 1024;
+  const size_t min_smem = lora::kExTmemCols > 256 ? 116 * 1024 : kTmemCtaMinSmem;
   if (smem < min_smem) smem = min_smem;
 
   const int64_t n_tot = a.slices.off[a.S] - a.slices.off[0];
@@ -472,6 +526,72 @@ lora_status expand_tc(const lora::ExpandArgs& a, lora_dtype dt, const Grouping& 
   cfg.stream = st;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, lora::expand_tc_kernel<E>, P);
   ++g_launches;
+  g_last_path = LORA_PATH_TENSOR | (P.vseg_indptr ? LORA_PATH_GROUPED : 0);
+  return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+}
+
+// Element-aligned tensor-core expand (expand_unaligned_tc.cuh): any 2-byte
+// alignment, leading dimension and slice layout, r <= 64.  *launched says
+// whether it ran (else the CUDA-core kernel takes the call).
+template <class E>
+lora_status expand_unaligned_tc(const lora::ExpandArgs& a, lora_dtype dt, const Grouping& g,
+                                const DeviceFacts& dev, cudaStream_t st, bool& launched) {
+  launched = false;
+  const int64_t n_tot = a.slices.off[a.S] - a.slices.off[0];
+  if (a.r > 64 || static_cast<int64_t>(a.L) * n_tot >= (int64_t(1) << 31) || a.tok >= (1 << 30))
+    return LORA_OK;
+  lora::ExpandUnalignedParams P;
+  std::memset(&P, 0, sizeof(P));
+  P.a = a;
+  P.row_list = g.row_list;
+  P.vseg_indptr = g.vseg_indptr;
+  P.nvseg = g.vseg_indptr ? g.nvseg : a.nseg;
+  P.rpad = a.r <= 16 ? 16 : (a.r <= 32 ? 32 : 64);
+  P.sw_layout = P.rpad == 16 ? 6u : (P.rpad == 32 ? 4u : 2u);
+  P.rin_bytes = lora::kExBM * P.rpad * 2;
+  P.btile_bytes = lora::kExBN * P.rpad * 2;
+  int tiles = 0;
+  for (int q = 0; q < a.S; ++q) {
+    P.tile_prefix[q] = tiles;
+    tiles += (a.slices.off[q + 1] - a.slices.off[q] + lora::kExBN - 1) / lora::kExBN;
+  }
+  for (int q = a.S; q <= LORA_MAX_SLICES; ++q) P.tile_prefix[q] = tiles;
+  if (tiles == 0) {
+    launched = true;
+    return LORA_OK;
+  }
+  P.tiles_total = tiles;
+  P.idesc = lora::make_idesc_f16(dt == LORA_BF16 ? 1 : 0, lora::kExBM, lora::kExBN);
+  P.stage_bytes = static_cast<uint32_t>(
+      round_up(lora::kEuRawBase + static_cast<int>(P.btile_bytes) + lora::kExBM * lora::kEuStageRow,
+               1024));
+  const size_t fixed = lora::kExStageBytes + static_cast<size_t>(a.S) * P.rin_bytes +
+                       4 * lora::kExBM + 1024 + 16;
+  auto total = [&](int nb) {
+    return static_cast<size_t>(nb) * P.stage_bytes + fixed + 8 * (3 * nb + 6);
+  };
+  P.stages = 2;
+  while (P.stages < 4 && total(P.stages + 1) <= 225 * 1024) ++P.stages;
+  if (total(P.stages) > 225 * 1024) return LORA_OK;
+  const size_t smem = std::max<size_t>(total(P.stages), 120 * 1024);  // one CTA per SM
+
+  const long slots = lora::num_piece_slots(a.tok, P.nvseg, lora::kExBM);
+  const long target = dev.sms;
+  long tpc = (slots * tiles + target - 1) / target;
+  if (tpc < 1) tpc = 1;
+  if (tpc > tiles) tpc = tiles;
+  P.tiles_per_cta = static_cast<int>(tpc);
+  const long ncg = (tiles + tpc - 1) / tpc;
+  if (slots * ncg >= (1L << 31)) return LORA_OK;
+
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(slots * ncg));
+  cfg.blockDim = dim3(lora::kExThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, lora::expand_unaligned_kernel<E>, P);
+  ++g_launches;
+  launched = true;
   g_last_path = LORA_PATH_TENSOR | (P.vseg_indptr ? LORA_PATH_GROUPED : 0);
   return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
 }
@@ -539,7 +659,7 @@ lora_status fused_tc(const lora::ShrinkArgs& sa, const lora::ExpandArgs& ea, lor
   // after the shrink, its ring holds further expand stages (8 in all at most)
   P.xstages = std::min(8, P.base_stages + static_cast<int>(static_cast<size_t>(P.stages) *
                                                            P.stage_bytes / lora::kExStageBytes));
-  // at least 120 KB, so that two CTAs never share an SM (and its TMEM)
+  // at least 120 KB: one CTA per SM
   const size_t smem = std::max<size_t>(total(P.stages), 120 * 1024);
 
   // cluster size: the largest of 16, 8, 4 CTAs for which every slot's cluster
@@ -698,6 +818,17 @@ lora_status lora_expand(const void* in_r, int64_t ld_in, const void* B_stack,
     if (gs != LORA_OK) return gs;
     return dtype == LORA_BF16 ? expand_tc<lora::Bf16>(a, dtype, g, *dev, st)
                               : expand_tc<lora::Fp16>(a, dtype, g, *dev, st);
+  }
+  {
+    Grouping g;
+    const lora_status gs =
+        maybe_group(seg_indptr, weight_indices, tok, nseg, L, workspace, workspace_bytes, st, g);
+    if (gs != LORA_OK) return gs;
+    bool launched = false;
+    const lora_status us = dtype == LORA_BF16
+                               ? expand_unaligned_tc<lora::Bf16>(a, dtype, g, *dev, st, launched)
+                               : expand_unaligned_tc<lora::Fp16>(a, dtype, g, *dev, st, launched);
+    if (us != LORA_OK || launched) return us;
   }
   return dtype == LORA_BF16 ? expand_general<lora::Bf16>(a, st)
                             : expand_general<lora::Fp16>(a, st);
@@ -984,7 +1115,8 @@ extern "C" lora_status lora_shrink_expand(
   const DeviceFacts* dev = device_facts();
   if (!dev) return LORA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (shrink_tc_eligible(sa) && expand_tc_eligible(ea) && tab.off[S] > tab.off[0]) {
+  if (shrink_tc_eligible(sa) && shrink_tc_aligned(sa) && expand_tc_eligible(ea) &&
+      tab.off[S] > tab.off[0]) {
     bool launched = false;
     const lora_status fs = dtype == LORA_BF16
                                ? fused_tc<lora::Bf16>(sa, ea, dtype, *dev, st, launched)
@@ -1044,8 +1176,8 @@ lora_status base_expand_tc(const lora::BaseExpandArgs& a, const void* W, int64_t
   P.stages = 2;
   while (P.stages < 6 && total(P.stages + 1) <= cap) ++P.stages;
   if (total(P.stages) > 225 * 1024) return LORA_ERR_UNSUPPORTED;
-  // at least 80 KB: never more than two CTAs (2 x 256 TMEM columns) on an SM
-  const size_t smem = std::max<size_t>(total(P.stages), 80 * 1024);
+  // never more than two CTAs (2 x 256 TMEM columns) on an SM
+  const size_t smem = std::max<size_t>(total(P.stages), kTmemCtaMinSmem);
 
   const int64_t n_tot = a.slices.off[a.S] - a.slices.off[0];
   if (!encode_2d(&P.tmap_W, dt, W, a.K, static_cast<uint64_t>(n_tot),

@@ -20,11 +20,12 @@
 //    thread) and round each valid column (j < r of every slice) once.
 //
 // Split-K: for small token counts the K range is split over the CTAs of a
-// thread-block cluster (grid = pieces x C, cluster = C CTAs along K).  Each
-// CTA leaves its fp32 partial in its own shared memory; after a cluster
-// barrier CTA c sums rows [c*128/C, (c+1)*128/C) over all C partials through
-// distributed shared memory, in rank order (deterministic), and writes them.
-// No global scratch and no atomics.
+// thread-block cluster (grid = pieces x C, cluster = C CTAs along K).  CTA c
+// owns rows [c*128/C, (c+1)*128/C) of the piece: every CTA pushes each of its
+// fp32 partial rows into the receive buffer of the row's owner with st.async
+// (distributed shared memory, completion counted in bytes on the owner's
+// mbarrier), and the owner sums the C partials of its rows in rank order
+// (deterministic) and writes them.  No global scratch and no atomics.
 #pragma once
 
 #include "common.cuh"
@@ -34,6 +35,13 @@
 
 #ifndef LORA_SHRINK_INTERLEAVE
 #define LORA_SHRINK_INTERLEAVE 1
+#endif
+// L2 hints of the x gather (sm100.cuh, cp_async_16_hint)
+#ifndef LORA_X_PREFETCH
+#define LORA_X_PREFETCH 0
+#endif
+#ifndef LORA_X_EVICT_FIRST
+#define LORA_X_EVICT_FIRST 1
 #endif
 
 namespace lora {
@@ -61,12 +69,25 @@ struct ShrinkTcParams {
   int csplit;                  // CTAs per cluster (K splits)
   uint32_t idesc;
   uint32_t stage_bytes;
+  int vec_out;                 // out_r 16-byte aligned with ld_out % 8 == 0
+  int recv_in_ring;            // split-K partials received in the (then idle) stage ring
 };
 
-// NSUB: 64-K sub-tiles per stage (stage K width = 64 * NSUB)
-template <class E, int NSUB>
+// Row staging of the element-aligned variant: the 16-byte blocks that cover
+// one row's 64 elements of a stage (at most 9), 144 bytes per row, so that
+// eight consecutive rows fall in eight different bank groups.
+constexpr int kRawRow = 144;
+
+// NSUB: 64-K sub-tiles per stage (stage K width = 64 * NSUB).
+// AL: x and A rows are 16-byte aligned with K % 8 == 0 (x rows by 16-byte
+// cp.async, A by TMA).  Otherwise (any 2-byte alignment, any K; NSUB = 1) each
+// producer thread copies the aligned 16-byte blocks that cover its own x row
+// (and A row) into a staging area of the stage, then shifts them into the
+// swizzled layout the MMA reads, zero-filling past K.
+template <class E, int NSUB, bool AL>
 __global__ void __launch_bounds__(kTcThreads, 1)
 shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
+  static_assert(AL || NSUB == 1, "the element-aligned stage is 64 K wide");
   constexpr int kTcNSub = NSUB;
   constexpr int kTcBK = NSUB * kTcAtomK;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -81,27 +102,39 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
                                              ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t x_bytes = kTcNSub * kTcBM * 128;  // kTcNSub sub-tiles of 128 rows x 128 B
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.stages * P.stage_bytes);
+  // split-K receive buffer: [C sources][128/C rows][npad] fp32, after the
+  // ring, or in the ring itself once every CTA of the cluster has finished its
+  // MMAs (when a separate buffer would leave too few stages)
+  float* recv = reinterpret_cast<float*>(smem + (P.recv_in_ring ? 0 : P.stages * P.stage_bytes));
+  const uint32_t recv_bytes = P.csplit > 1 && !P.recv_in_ring ? kTcBM * P.npad * 4 : 0;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.stages * P.stage_bytes + recv_bytes);
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * P.stages;
   const uint32_t done_bar = empty0 + 8 * P.stages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * P.stages + 1);
-  int64_t* xrow_tok = reinterpret_cast<int64_t*>(bars + 2 * P.stages + 2);  // [128] x row index
+  const uint32_t recv_bar = done_bar + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * P.stages + 2);
+  int64_t* xrow_tok = reinterpret_cast<int64_t*>(bars + 2 * P.stages + 3);  // [128] x row index
 
   // barriers and TMEM first, so that their latency overlaps the table reads
   if (tid == 0) {
     for (int s = 0; s < P.stages; ++s) {
-      mbar_init(full0 + 8 * s, kTcBM + 1);
+      mbar_init(full0 + 8 * s, AL ? kTcBM + 1 : kTcBM);  // + the A transfer (TMA)
       mbar_init(empty0 + 8 * s, 1);
     }
     mbar_init(done_bar, 1);
+    mbar_init(recv_bar, 1);
     fence_mbar_init();
-    tma_prefetch_desc(&P.tmap_A);
+    if (AL) tma_prefetch_desc(&P.tmap_A);
   }
   if (warp == 4) {
     tmem_alloc(smem_u32(tmem_slot), P.tmem_cols);
     tmem_relinquish();
   }
+  // the receive barrier must be initialised before any peer pushes into it:
+  // arrive now, wait just before the first push (a receive buffer in the ring
+  // has a cluster barrier of its own after the MMAs instead)
+  const bool early_arrive = P.csplit > 1 && !P.recv_in_ring;
+  if (early_arrive) cluster_arrive_relaxed();
 
   // ---- piece of this cluster (identical in all its CTAs).  Rows of a block
   // slot start at slot*128, so their tokens are fetched while the tables are read.
@@ -117,6 +150,7 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
   if (!find_piece_warp(indptr, P.vseg_indptr ? nullptr : p.weight_indices, nullptr, P.nvseg,
                        p.L, p.tok, kTcBM, slot, pc)) {
     // no rows here (the same answer in every CTA of the cluster): give TMEM back
+    if (early_arrive) cluster_wait();  // pairs the arrive above
     tc_fence_before();
     __syncthreads();
     if (warp == 4) {
@@ -127,6 +161,8 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
   }
   const int rows = pc.hi - pc.lo;
   const int adapter = pc.adapter;
+  const int R = kTcBM / P.csplit;  // rows owned by each CTA of the cluster
+  const int nmine = max(0, min(R, rows - split * R));
 
   // K blocks of this CTA.  Interleaved over the cluster (CTA c takes blocks
   // c, c+C, c+2C, ...), so the C co-scheduled CTAs of a piece read C adjacent
@@ -140,6 +176,25 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
   const int nk = max(0, min(P.nkb, kb0 + P.kb_per) - kb0);
 #define LORA_KB(i) (kb0 + (i))
 #endif
+
+  // The adapter's A blocks of the first stages do not depend on the x rows:
+  // request them now, before the row tokens are known.
+  const uint32_t a_sub = P.npad * 128;  // one 64-K sub-tile of A
+  const uint32_t a_bytes = kTcNSub * a_sub;
+  const int pre_a = AL ? min(nk, P.stages) : 0;
+  if (tid == 0) {
+    for (int i = 0; i < pre_a; ++i) {
+      const uint32_t as = sbase + i * P.stage_bytes + x_bytes;
+      const int k0 = LORA_KB(i) * kTcBK;
+      mbar_arrive_expect_tx(full0 + 8 * i, a_bytes);
+#pragma unroll
+      for (int sub = 0; sub < kTcNSub; ++sub)
+        tma_load_2d(as + sub * a_sub, &P.tmap_A, full0 + 8 * i, k0 + sub * kTcAtomK,
+                    adapter * p.S * p.rs);
+    }
+    if (P.csplit > 1)
+      mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(P.csplit * nmine * P.npad * 4));
+  }
 
   if (tid < kTcBM) {
     const int m = tid;
@@ -157,7 +212,97 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
 
-  if (warp < 4) {
+  if (!AL && warp < 4) {
+    // =========================== producer, element-aligned rows
+    // Thread m stages x row m and A rows m and m + 128 of the stage's 64 K
+    // columns: copy the covering 16-byte blocks (cp.async through L1, one row
+    // per thread), and once they have landed (lagged like the aligned path)
+    // shift them into the swizzled K-major layout, zero past K.
+    const int m = tid;
+    const uint32_t raw_x = x_bytes + P.npad * 128;     // offsets inside a stage
+    const uint32_t raw_a = raw_x + kTcBM * kRawRow;
+    const uint16_t* rowp[3];
+    bool rowok[3];
+    uint32_t rawo[3], dsto[3];
+    int rown[3];
+    rowp[0] = p.x + xrow_tok[m] * p.ld_x;
+    rowok[0] = m < rows;
+    rawo[0] = raw_x + m * kRawRow;
+    dsto[0] = m * 128;
+    rown[0] = m;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int n = m + 128 * h;
+      rowok[1 + h] = n < P.npad && n < p.S * p.rs;
+      rowp[1 + h] = p.A + (static_cast<int64_t>(adapter) * p.S * p.rs + (rowok[1 + h] ? n : 0)) *
+                              p.K;
+      rawo[1 + h] = raw_a + n * kRawRow;
+      dsto[1 + h] = x_bytes + n * 128;
+      rown[1 + h] = n;
+    }
+    auto issue_rows = [&](uint32_t st, int k0) {
+      const int nv = min(kTcAtomK, p.K - k0);
+#pragma unroll
+      for (int h = 0; h < 3; ++h) {
+        if (!rowok[h]) continue;
+        const uintptr_t a = reinterpret_cast<uintptr_t>(rowp[h] + k0);
+        const uintptr_t a0 = a & ~static_cast<uintptr_t>(15);
+        const uintptr_t a1 = (a + 2 * nv + 15) & ~static_cast<uintptr_t>(15);
+        for (uintptr_t b = a0; b < a1; b += 16)
+          cp_async_16_ca(st + rawo[h] + static_cast<uint32_t>(b - a0),
+                         reinterpret_cast<const void*>(b));
+      }
+    };
+    auto realign_rows = [&](int j) {
+      const uint32_t st = sbase + (j % P.stages) * P.stage_bytes;
+      const uint8_t* stp = smem + (j % P.stages) * P.stage_bytes;
+      const int k0 = LORA_KB(j) * kTcBK;
+      const int nv = min(kTcAtomK, p.K - k0);
+#pragma unroll
+      for (int h = 0; h < 3; ++h) {
+        if (!rowok[h]) continue;
+        const int off = static_cast<int>(reinterpret_cast<uintptr_t>(rowp[h] + k0) & 15);
+        const uint4* raw = reinterpret_cast<const uint4*>(stp + rawo[h]);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int keep = min(8, max(0, nv - 8 * c));
+          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+          if (keep > 0) {
+            const int pos = off + 16 * c, blk = pos >> 4, sh = pos & 15;
+            const uint4 w0 = raw[blk];
+            const uint4 w1 = (sh != 0 && blk < 8) ? raw[blk + 1] : make_uint4(0u, 0u, 0u, 0u);
+            v = keep_elems(bytes_at(w0, w1, sh), keep);
+          }
+          *reinterpret_cast<uint4*>(const_cast<uint8_t*>(stp) + dsto[h] +
+                                    ((c ^ (rown[h] & 7)) << 4)) = v;
+        }
+      }
+      (void)st;
+    };
+    const int lag = P.stages - 1;
+    for (int i = 0; i < nk && ok; ++i) {
+      const int s = i % P.stages;
+      if (i >= P.stages) ok = mbar_wait(empty0 + 8 * s, ((i / P.stages) - 1) & 1);
+      if (!ok) break;
+      issue_rows(sbase + s * P.stage_bytes, LORA_KB(i) * kTcBK);
+      cp_async_commit();
+      if (i >= lag) {
+        cp_async_wait_dyn(lag);
+        realign_rows(i - lag);
+        fence_proxy_async_smem();
+        mbar_arrive(full0 + 8 * ((i - lag) % P.stages));
+      }
+    }
+    if (ok) {
+      for (int i = max(0, nk - lag); i < nk; ++i) {
+        cp_async_wait_dyn(nk - 1 - i);
+        realign_rows(i);
+        fence_proxy_async_smem();
+        mbar_arrive(full0 + 8 * (i % P.stages));
+      }
+    }
+    cp_async_wait<0>();
+  } else if (warp < 4) {
     // =========================== producer: gather x rows and the A block
     // A stage holds NSUB sub-tiles of 16-byte chunks; chunk u = j*128 + tid ->
     // row u / (8*NSUB), chunk u % (8*NSUB).  The chunk column of a thread is the
@@ -170,21 +315,20 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
     const int rr = tid / CPR;                     // ... and first row
     const int wrow0 = (tid & ~31) / CPR;          // first row of this warp
     const uint32_t sub_off = (cc >> 3) * (kTcBM * 128);  // x sub-tile of this chunk
-    const uint32_t a_sub = P.npad * 128;  // one 64-K sub-tile of A
-    const uint32_t a_bytes = kTcNSub * a_sub;
     // gathered x row of each of this thread's CPR rows (rows past the piece are
     // never read)
     const uint16_t* xr[CPR];
 #pragma unroll
     for (int j = 0; j < CPR; ++j) xr[j] = p.x + xrow_tok[rr + j * RSTEP] * p.ld_x;
     const int lag = P.stages - 1;
+    const uint64_t pol = LORA_X_EVICT_FIRST ? policy_evict_first() : 0;
     for (int i = 0; i < nk && ok; ++i) {
       const int s = i % P.stages;
       if (i >= P.stages) ok = mbar_wait(empty0 + 8 * s, ((i / P.stages) - 1) & 1);
       if (!ok) break;
       const uint32_t xs = sbase + s * P.stage_bytes;
       const int k0 = LORA_KB(i) * kTcBK;
-      if (tid == 0) {
+      if (tid == 0 && i >= pre_a) {
         mbar_arrive_expect_tx(full0 + 8 * s, a_bytes);
 #pragma unroll
         for (int sub = 0; sub < kTcNSub; ++sub)
@@ -199,8 +343,9 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
         const int row = rr + j * RSTEP;
         const bool in = k_in && row < rows;
         const uint32_t dst = xs + sub_off + row * 128 + (((cc & 7) ^ (row & 7)) << 4);
-        cp_async_16(dst, in ? static_cast<const void*>(xr[j] + k) : static_cast<const void*>(p.x),
-                    in ? 16u : 0u);
+        cp_async_16_hint<LORA_X_PREFETCH, LORA_X_EVICT_FIRST != 0>(
+            dst, in ? static_cast<const void*>(xr[j] + k) : static_cast<const void*>(p.x),
+            in ? 16u : 0u, pol);
       };
       if (rows >= kTcBM) {
 #pragma unroll
@@ -260,18 +405,51 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
   }
 
   // =========================== epilogue (warps 0-3: one accumulator row per thread)
-  // Split-K partials reuse the stage ring as [128][npad + 4] fp32: 16-byte rows
-  // whose stride (4 or 20 words mod 32) keeps the row-per-thread 16-byte
-  // stores free of bank conflicts.
-  float* part = reinterpret_cast<float*>(smem);
-  const int pstride = P.npad + 4;
+  const int nvalid = p.S * p.rs;
+  // columns [n0, n0+8) of output row `orow_i`, rounded once: one 16-byte store
+  // when all eight are valid outputs (j < r) and the row is 16-byte aligned,
+  // otherwise element by element
+  auto store8 = [&](int orow_i, int n0, const float* v) {
+    uint16_t* orow = p.out + static_cast<int64_t>(orow_i) * p.ld_out;
+    const bool full = P.vec_out && n0 + 8 <= nvalid && (n0 % p.rs) + 8 <= p.r;
+    if (full) {
+      uint4 w;
+      w.x = E::f2_to_u32(v[0], v[1]);
+      w.y = E::f2_to_u32(v[2], v[3]);
+      w.z = E::f2_to_u32(v[4], v[5]);
+      w.w = E::f2_to_u32(v[6], v[7]);
+      *reinterpret_cast<uint4*>(orow + n0) = w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int n = n0 + i;
+        if (n < nvalid && (n % p.rs) < p.r) orow[n] = E::f32_to_bits(v[i]);
+      }
+    }
+  };
   if (warp < 4) {
     if (ok) ok = mbar_wait(done_bar, 0);
     ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+  }
+  if (P.csplit > 1) {
+    if (early_arrive) cluster_wait();  // every receive barrier of the cluster is initialised
+    else cluster_sync();  // every CTA's MMAs are done: its ring may receive partials
+  }
+  if (warp < 4) {
     tc_fence_after();
     const int m = tid;
     const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const int nvalid = p.S * p.rs;
+    // split-K: row m goes to CTA m / R of the cluster, into the slot of this
+    // CTA's rank
+    const int owner = m / R;
+    const uint32_t rdst = P.csplit > 1
+        ? mapa_shared(smem_u32(recv) + 4u * static_cast<uint32_t>((split * R + m % R) * P.npad),
+                      owner)
+        : 0u;
+    const uint32_t rbar = P.csplit > 1 ? mapa_shared(recv_bar, owner) : 0u;
+    const int orow_i = P.csplit == 1 && m < rows
+        ? (P.row_list ? clampi(__ldg(P.row_list + pc.lo + m), 0, p.tok - 1) : pc.lo + m)
+        : 0;
     for (int c0 = 0; c0 < P.npad; c0 += 16) {
       float v[16];
       if (nk > 0 && ok) {
@@ -281,68 +459,42 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = 0.f;
       }
-      if (P.csplit == 1) {
-        if (m < rows && ok) {
-          const int orow_i = P.row_list ? clampi(__ldg(P.row_list + pc.lo + m), 0, p.tok - 1)
-                                        : pc.lo + m;
-          uint16_t* orow = p.out + static_cast<int64_t>(orow_i) * p.ld_out;
+      if (m < rows && ok) {
+        if (P.csplit == 1) {
+          store8(orow_i, c0, v);
+          store8(orow_i, c0 + 8, v + 8);
+        } else {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int n = c0 + i;
-            if (n < nvalid && (n % p.rs) < p.r) orow[n] = E::f32_to_bits(v[i]);
-          }
+          for (int k = 0; k < 4; ++k)
+            st_async_v4(rdst + 4u * static_cast<uint32_t>(c0 + 4 * k),
+                        make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]), rbar);
         }
-      } else {
-        float4* dst = reinterpret_cast<float4*>(part + m * pstride + c0);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
       }
     }
     tc_fence_before();
   }
 
   if (P.csplit > 1) {
-    cluster_sync();  // every partial of the cluster is in shared memory
-    // CTA `split` owns rows [split*R, (split+1)*R); a thread sums one 4-column
-    // group over all C partials: the C remote 16-byte loads are issued back to
-    // back and only then added, in rank order (deterministic).
-    const int R = kTcBM / P.csplit;
-    const int r0 = split * R;
-    const int ng = P.npad / 4;
-    const int nvalid = p.S * p.rs;
-    const uint32_t pbase = smem_u32(part);
-    for (int e = tid; e < R * ng; e += kTcThreads) {
-      const int row = r0 + e / ng;
-      const int g = e % ng;
-      if (row >= rows) continue;
-      const uint32_t off = pbase + 4u * static_cast<uint32_t>(row * pstride + 4 * g);
-      float4 pv[16];
-#pragma unroll
-      for (int q = 0; q < 16; ++q)
-        if (q < P.csplit) pv[q] = ld_dsmem_v4(mapa_shared(off, q));
-      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        if (q < P.csplit) {
-          sum.x += pv[q].x;
-          sum.y += pv[q].y;
-          sum.z += pv[q].z;
-          sum.w += pv[q].w;
-        }
+    // rows [split*R, split*R + nmine) of the piece: the C partials of each
+    // 8-column group summed in rank order (deterministic), rounded once
+    if (ok) ok = mbar_wait(recv_bar, 0);
+    const int ng = P.npad / 8;
+    for (int e = tid; e < nmine * ng && ok; e += kTcThreads) {
+      const int lr = e / ng, n0 = 8 * (e % ng);
+      float sum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int src = 0; src < P.csplit; ++src) {
+        const float4* pp = reinterpret_cast<const float4*>(recv + (src * R + lr) * P.npad + n0);
+        const float4 a0 = pp[0], a1 = pp[1];
+        sum[0] += a0.x; sum[1] += a0.y; sum[2] += a0.z; sum[3] += a0.w;
+        sum[4] += a1.x; sum[5] += a1.y; sum[6] += a1.z; sum[7] += a1.w;
       }
+      const int row = split * R + lr;
       const int orow_i = P.row_list ? clampi(__ldg(P.row_list + pc.lo + row), 0, p.tok - 1)
                                     : pc.lo + row;
-      uint16_t* orow = p.out + static_cast<int64_t>(orow_i) * p.ld_out;
-      const float sv[4] = {sum.x, sum.y, sum.z, sum.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int n = 4 * g + k;
-        if (ok && n < nvalid && (n % p.rs) < p.r) orow[n] = E::f32_to_bits(sv[k]);
-      }
+      store8(orow_i, n0, sum);
     }
-    // peers are done reading this CTA's partial (their loads have returned:
-    // the sums above used them), so the arrive needs no release ordering
+    // a CTA leaves only after its peers: none of them is still writing into it
+    // (each waited for its own receive), and none still needs this CTA
     cluster_sync_relaxed();
   }
 

@@ -98,6 +98,72 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint3
                : "memory");
 }
 
+// The same copy of a streamed operand, with L2 hints: PF = bytes the L2 may
+// fetch around the copied 16 (0, 64, 128 or 256); EF = mark the line
+// evict-first under policy `pol` (from policy_evict_first), for data read once.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+template <int PF, bool EF>
+__device__ __forceinline__ void cp_async_16_hint(uint32_t dst, const void* src,
+                                                 uint32_t src_bytes, uint64_t pol) {
+  if constexpr (EF) {
+    if constexpr (PF == 256)
+      asm volatile("cp.async.cg.shared.global.L2::cache_hint.L2::256B [%0], [%1], 16, %2, %3;" ::
+                       "r"(dst), "l"(src), "r"(src_bytes), "l"(pol) : "memory");
+    else if constexpr (PF == 128)
+      asm volatile("cp.async.cg.shared.global.L2::cache_hint.L2::128B [%0], [%1], 16, %2, %3;" ::
+                       "r"(dst), "l"(src), "r"(src_bytes), "l"(pol) : "memory");
+    else
+      asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst),
+                   "l"(src), "r"(src_bytes), "l"(pol) : "memory");
+  } else {
+    (void)pol;
+    if constexpr (PF == 256)
+      asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                   "r"(src_bytes) : "memory");
+    else if constexpr (PF == 128)
+      asm volatile("cp.async.cg.shared.global.L2::128B [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                   "r"(src_bytes) : "memory");
+    else
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                   "r"(src_bytes) : "memory");
+  }
+}
+
+// 16-byte copy global -> shared through L1 (both addresses 16-byte aligned).
+__device__ __forceinline__ void cp_async_16_ca(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// The 16 bytes starting `sh` bytes (even, 0..14) into the 32 bytes a:b.
+__device__ __forceinline__ uint4 bytes_at(uint4 a, uint4 b, int sh) {
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  const int q = sh >> 2, r = (sh & 3) * 8;
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t lo = q == 0 ? w[i] : q == 1 ? w[i + 1] : q == 2 ? w[i + 2] : w[i + 3];
+    const uint32_t hi = q == 0 ? w[i + 1] : q == 1 ? w[i + 2] : q == 2 ? w[i + 3] : w[i + 4];
+    o[i] = __funnelshift_r(lo, hi, r);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Keeps the first n (0..8) 16-bit elements of v and zeroes the others.
+__device__ __forceinline__ uint4 keep_elems(uint4 v, int n) {
+  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = 2 * i;
+    w[i] = e + 2 <= n ? w[i] : (e + 1 == n ? (w[i] & 0xFFFFu) : 0u);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // Arrives on the mbarrier once all of this thread's prior cp.async copies have
 // landed; the arrival is one of the barrier's expected arrivals (.noinc).
 __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
@@ -278,6 +344,26 @@ __device__ __forceinline__ void cluster_sync() {
 __device__ __forceinline__ void cluster_sync_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" :::
                    "memory");
+}
+
+// Split cluster barrier: arrive early (no ordering of earlier memory accesses
+// beyond what a preceding fence gives), wait later (acquire).
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// 16-byte store into the shared memory of a CTA of this cluster that completes
+// `16` transaction bytes on that CTA's mbarrier (both addresses from mapa).
+__device__ __forceinline__ void st_async_v4(uint32_t caddr, float4 v, uint32_t cbar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, "
+      "[%5];" ::"r"(caddr),
+      "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(cbar)
+      : "memory");
 }
 
 __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {

@@ -90,3 +90,11 @@ def test_base_expand_misaligned_is_unsupported():
                               [int(v) for v in p.slice_offsets],
                               torch.from_numpy(p.scalings).cuda(), out, rank=p.r)
     assert e.value.status == lora.LORA_ERR_UNSUPPORTED
+
+
+def test_base_expand_full_qkv_shape():
+    # the projection at the qkv workload's K = 4096 with its 4096/1024/1024
+    # slices and eight adapters of rank 16, at a token count the oracle
+    # finishes in seconds (a few 128-row pieces per segment, ragged)
+    p = make_problem("qkv", seed=86, tok=256)
+    run(p, make_base_weight(p, 86))

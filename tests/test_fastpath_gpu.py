@@ -22,12 +22,67 @@ def test_aligned_inputs_take_the_tensor_core_path():
     assert lora.last_path() & T
 
 
-def test_misaligned_inputs_take_the_general_path():
+def test_misaligned_inputs_take_the_tensor_core_path_too():
+    # element-aligned rows are staged and shifted for the tensor cores
     p = make_problem("tail", seed=21, tok=100)
     check_shrink(p)
-    assert lora.last_path() == GEN
+    assert lora.last_path() & T
     check_expand(p)
-    assert lora.last_path() == GEN
+    assert lora.last_path() & T
+
+
+# element-aligned expand: pointer offsets, odd leading dimensions, odd slice
+# starts and widths, odd ranks of every padding class, grouped schedule
+@pytest.mark.parametrize("mis", [1, 2, 3, 5, 7])
+def test_expand_element_aligned_offsets(mis):
+    p = make_problem("qkv", seed=50 + mis, tok=300, K=64, slices=[200 + mis, 131, 67],
+                     r=13, rs=16, misalign=mis, ld_pad=mis, col_lead=mis)
+    check_expand(p)
+    assert lora.last_path() & T
+
+
+@pytest.mark.parametrize("r,rs", [(5, 7), (16, 16), (29, 33), (64, 64)])
+def test_expand_element_aligned_ranks(r, rs):
+    p = make_problem("qkv", seed=60 + r, tok=257, K=64, slices=[129, 7, 260], r=r, rs=rs,
+                     misalign=1, ld_pad=3, col_lead=1)
+    check_expand(p)
+    assert lora.last_path() & T
+
+
+def test_expand_element_aligned_grouped_zero_scaling_and_lead_trail():
+    p = make_problem("many_small", seed=70, tok=900, nseg=120, K=64, slices=[250, 70, 70],
+                     misalign=3, lead=9, trail=4, col_lead=5)
+    sc = p.scalings.copy()
+    sc[::3] = 0.0
+    check_expand(p, workspace=True, scalings=sc)
+    assert lora.last_path() & G and lora.last_path() & T
+
+
+# element-aligned shrink: every pointer offset (elements past a 16-byte
+# boundary), odd K and leading dimensions, odd ranks, split-K and grouped
+@pytest.mark.parametrize("mis", [1, 2, 3, 4, 5, 6, 7])
+def test_shrink_element_aligned_offsets(mis):
+    p = make_problem("qkv", seed=30 + mis, tok=300, K=1000 + mis, slices=[64, 32, 32],
+                     r=13, rs=16, misalign=mis, ld_pad=mis)
+    check_shrink(p)
+    assert lora.last_path() & T
+
+
+@pytest.mark.parametrize("K", [1, 7, 63, 65, 129, 3583])
+def test_shrink_element_aligned_k_tails(K):
+    p = make_problem("qkv", seed=40, tok=150, K=K, slices=[64, 64], r=8, rs=8, misalign=1)
+    check_shrink(p)
+    assert lora.last_path() & T
+
+
+def test_shrink_element_aligned_grouped_and_split():
+    p = make_problem("many_small", seed=41, tok=900, nseg=120, K=777, slices=[256, 64, 64],
+                     misalign=3)
+    check_shrink(p, workspace=True)
+    assert lora.last_path() & G and lora.last_path() & T
+    p = make_problem("qkv", seed=42, tok=40, K=4093, misalign=5)
+    check_shrink(p)
+    assert lora.last_path() & T and lora.last_path() & SPLIT
 
 
 def test_many_segments_with_workspace_are_grouped():

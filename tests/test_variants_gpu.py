@@ -44,7 +44,11 @@ def test_sgemm_lora_a(dtype):
 @pytest.mark.parametrize("dtype", ["bf16", "fp16"])
 def test_expand_variants(op, dtype):
     slices = {"sgemm_b": [640], "qkv_b": [512, 128, 128], "gate_up_b": [384, 384]}[op]
-    p = identity(make_problem("qkv", seed=52, tok=300, K=64, slices=slices, dtype=dtype))
+    # rows before and after the segments (and, for the op with explicit
+    # offsets, columns before slice 0) that nothing may touch
+    extra = dict(lead=7, trail=5, col_lead=16 if op == "qkv_b" else 0)
+    p = identity(make_problem("qkv", seed=52, tok=300, K=64, slices=slices, dtype=dtype,
+                              **extra))
     ref = oracle.expand_problem(p)
     base = dev(p.base, dtype)
     args = (dev(p.in_r, dtype), dev(p.B, dtype), torch.from_numpy(p.seg_indptr).cuda(),
@@ -56,7 +60,18 @@ def test_expand_variants(op, dtype):
         lora.qkv_lora_b_fwd(*args, p.slice_offsets.tolist(), sc, base, rank=p.r)
     else:
         lora.gate_up_lora_b_fwd(*args, sc, base, rank=p.r)
-    assert_close(bits_of(base), ref, dtype)
+    got = bits_of(base)
+    # write set, bit for bit: only the rows of the segments (zero-scaled
+    # adapters excluded) and the slice columns may change
+    touched = np.zeros(got.shape, dtype=bool)
+    off = p.slice_offsets
+    for s in range(p.nseg):
+        if p.scalings[p.weight_indices[s]] == 0.0:
+            continue
+        rows = np.arange(p.seg_indptr[s], p.seg_indptr[s + 1])
+        touched[np.ix_(rows, np.arange(off[0], off[-1]))] = True
+    assert np.array_equal(got[~touched], p.base[~touched]), f"{op} wrote outside its write set"
+    assert_close(got[touched], ref[touched], dtype)
 
 
 @pytest.mark.parametrize("nseg,tok", [(4, 500), (300, 300), (3000, 3000)])
