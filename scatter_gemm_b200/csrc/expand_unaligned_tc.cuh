@@ -23,7 +23,9 @@
 //     outside the tile's columns is written.
 // Warp roles (416 threads): warp 0 TMEM and MMA issue, warps 1-8 consumers as
 // in expand_tc.cuh; warps 9-11 stage base blocks, warp 12 stages and realigns
-// the B tiles (the four stage the rank activations first).  One CTA per SM.
+// the B tiles one tile ahead (the four stage the rank activations first, all
+// slices in one round trip, while the first base tiles are on their way).
+// One CTA per SM.
 #pragma once
 
 #include "common.cuh"
@@ -186,84 +188,108 @@ expand_unaligned_kernel(const __grid_constant__ ExpandUnalignedParams P) {
   if (warp >= 9) {
     // =========================== producers (128 threads)
     const int m = tid - 9 * 32;
-    // rank activations of row m, slice by slice, through a staging row in
-    // the (still unused) logical tile
-    {
-      int sr = pc.lo + (m < rows ? m : 0);
-      if (P.row_list) sr = clampi(__ldg(P.row_list + sr), 0, p.tok - 1);
-      uint8_t* raw = logical + m * kEuStageRow;
-      for (int q = 0; q < p.S; ++q) {
-        const uint16_t* src = p.in_r + static_cast<int64_t>(sr) * p.ld_in + q * p.rs;
-        if (m < rows) stage_blocks(smem_u32(raw), src, 2 * p.r);
-        cp_async_commit();
-        cp_async_wait<0>();
-        const int off = static_cast<int>(reinterpret_cast<uintptr_t>(src) & 15);
-        realign_row(rin_p + q * P.rin_bytes, m, P.rpad, raw, off, m < rows ? p.r : 0);
+    // base tile t into stage t % NB: block u = j*96 + i -> row u / 17, block u % 17
+    auto issue_base = [&](int t, int i) {
+      constexpr int kBaseThreads = 96;
+      int q, c0;
+      tile_info(t, q, c0);
+      const int ncols = min(kExBN, p.slices.off[q + 1] - c0);
+      const uint32_t st = sbase + (t % NB) * P.stage_bytes;
+      for (int u = i; u < kExBM * kEuRawBlocks; u += kBaseThreads) {
+        const int row = u / kEuRawBlocks, b = u % kEuRawBlocks;
+        if (row >= rows) break;  // u grows with the row
+        const uintptr_t a = reinterpret_cast<uintptr_t>(seg_addr(row, c0));
+        const uintptr_t a0 = a & ~static_cast<uintptr_t>(15);
+        const uintptr_t a1 = (a + 2 * ncols + 15) & ~static_cast<uintptr_t>(15);
+        const uintptr_t blk = a0 + 16 * static_cast<uintptr_t>(b);
+        if (blk < a1)
+          cp_async_16_ca(st + row * kEuRawRow + b * 16, reinterpret_cast<const void*>(blk));
       }
-      fence_proxy_async_smem();
-      mbar_arrive(rin_bar);
-    }
+      cp_async_arrive_noinc(xfull0 + 8 * (t % NB));
+      cp_async_commit();
+    };
+    // (1) the rank activations of row m, every slice at once: slice 0 staged
+    //     in the logical tile, slice q >= 1 in stage q-1's B staging area
+    //     (all still unused; the host keeps S <= stages + 1)
+    int sr = pc.lo + (m < rows ? m : 0);
+    if (P.row_list) sr = clampi(__ldg(P.row_list + sr), 0, p.tok - 1);
+    const uint16_t* rsrc = p.in_r + static_cast<int64_t>(sr) * p.ld_in;
+    auto rin_staging = [&](int q) {
+      return q == 0 ? logical + m * kEuStageRow
+                    : smem + (q - 1) * P.stage_bytes + kEuRawBase + P.btile_bytes +
+                          m * kEuStageRow;
+    };
+    if (m < rows)
+      for (int q = 0; q < p.S; ++q) stage_blocks(smem_u32(rin_staging(q)), rsrc + q * p.rs, 2 * p.r);
+    cp_async_commit();
+    // (2) the base warps send their first tiles out while those land
+    const int pre = warp != 12 ? min(NB, ntl) : 0;
+    for (int t = 0; t < pre; ++t) issue_base(t, tid - 9 * 32);
+    // (3) every group but the base tiles' has landed: realign the rank rows
+    cp_async_wait_dyn(pre);
+    for (int q = 0; q < p.S; ++q)
+      realign_row(rin_p + q * P.rin_bytes, m, P.rpad, rin_staging(q),
+                  static_cast<int>(reinterpret_cast<uintptr_t>(rsrc + q * p.rs) & 15),
+                  m < rows ? p.r : 0);
+    fence_proxy_async_smem();
+    mbar_arrive(rin_bar);
     if (warp == 12) {
-      // ---- B tiles (warp 12): rows m, m+32, m+64, m+96 of each tile, staged
-      //      and realigned; this warp issues no other copies, so waiting for
-      //      its own copies waits for nothing else
+      // ---- B tiles (warp 12): rows l, l+32, l+64, l+96 of each tile, staged
+      //      one tile ahead and realigned; this warp issues no other copies,
+      //      so waiting for its own copies waits for nothing else
       const int l = tid - 12 * 32;
+      ok = mbar_wait(rin_bar, 0);  // no B staging area holds rank rows any more
+      auto brow = [&](int c0, int k, bool& okk) {
+        const int n = l + 32 * k;  // output column c0 + n; past the last slice: zero
+        okk = c0 + n < p.slices.off[p.S];
+        return p.B + (static_cast<int64_t>(adapter) * n_tot + (okk ? c0 - off0 + n : 0)) * p.rs;
+      };
+      auto stage_b = [&](int t) {
+        int q, c0;
+        tile_info(t, q, c0);
+        const uint32_t st = sbase + (t % NB) * P.stage_bytes;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          bool okk;
+          const uint16_t* src = brow(c0, k, okk);
+          if (okk)
+            stage_blocks(st + kEuRawBase + P.btile_bytes + (l + 32 * k) * kEuStageRow, src,
+                         2 * p.r);
+        }
+        cp_async_commit();
+      };
+      if (ok && ntl > 0) stage_b(0);
       for (int t = 0; t < ntl && ok; ++t) {
         const int s = t % NB;
-        if (t >= NB) ok = mbar_wait(xempty0 + 8 * s, ((t / NB) - 1) & 1);
-        if (!ok) break;
+        cp_async_wait<0>();  // tile t's rows have landed (the only copies in flight)
         int q, c0;
         tile_info(t, q, c0);
         uint8_t* stp = smem + s * P.stage_bytes;
-        const uint32_t st = sbase + s * P.stage_bytes;
-        const uint16_t* bsrc[4];
-        bool bok[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int n = l + 32 * k;  // output column c0 + n
-          bok[k] = c0 + n < p.slices.off[p.S];  // past the last slice: zero
-          bsrc[k] = p.B + (static_cast<int64_t>(adapter) * n_tot + (bok[k] ? c0 - off0 + n : 0)) *
-                              p.rs;
-          if (bok[k]) stage_blocks(st + kEuRawBase + P.btile_bytes + n * kEuStageRow, bsrc[k],
-                                   2 * p.r);
-        }
-        cp_async_commit();
-        cp_async_wait<0>();
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
+          bool okk;
+          const uint16_t* src = brow(c0, k, okk);
           const int n = l + 32 * k;
           realign_row(stp + kEuRawBase, n, P.rpad,
                       stp + kEuRawBase + P.btile_bytes + n * kEuStageRow,
-                      static_cast<int>(reinterpret_cast<uintptr_t>(bsrc[k]) & 15),
-                      bok[k] ? p.r : 0);
+                      static_cast<int>(reinterpret_cast<uintptr_t>(src) & 15), okk ? p.r : 0);
         }
         fence_proxy_async_smem();
         mbar_arrive(bfull0 + 8 * s);
+        // the next tile's rows go out while this tile is multiplied
+        if (t + 1 < ntl) {
+          const int s1 = (t + 1) % NB;
+          if (t + 1 >= NB) ok = mbar_wait(xempty0 + 8 * s1, (((t + 1) / NB) - 1) & 1);
+          if (ok) stage_b(t + 1);
+        }
       }
     } else {
-      // ---- base blocks (warps 9-11): block u = j*96 + i -> row u / 17, block u % 17
-      const int i = tid - 9 * 32;
-      constexpr int kBaseThreads = 96;
-      for (int t = 0; t < ntl && ok; ++t) {
+      // ---- base blocks (warps 9-11), from tile `pre` on
+      for (int t = pre; t < ntl && ok; ++t) {
         const int s = t % NB;
         if (t >= NB) ok = mbar_wait(xempty0 + 8 * s, ((t / NB) - 1) & 1);
         if (!ok) break;
-        int q, c0;
-        tile_info(t, q, c0);
-        const int ncols = min(kExBN, p.slices.off[q + 1] - c0);
-        const uint32_t st = sbase + s * P.stage_bytes;
-        for (int u = i; u < kExBM * kEuRawBlocks; u += kBaseThreads) {
-          const int row = u / kEuRawBlocks, b = u % kEuRawBlocks;
-          if (row >= rows) break;  // u grows with the row
-          const uintptr_t a = reinterpret_cast<uintptr_t>(seg_addr(row, c0));
-          const uintptr_t a0 = a & ~static_cast<uintptr_t>(15);
-          const uintptr_t a1 = (a + 2 * ncols + 15) & ~static_cast<uintptr_t>(15);
-          const uintptr_t blk = a0 + 16 * static_cast<uintptr_t>(b);
-          if (blk < a1)
-            cp_async_16_ca(st + row * kEuRawRow + b * 16, reinterpret_cast<const void*>(blk));
-        }
-        cp_async_arrive_noinc(xfull0 + 8 * s);
-        cp_async_commit();
+        issue_base(t, tid - 9 * 32);
       }
     }
     cp_async_wait<0>();

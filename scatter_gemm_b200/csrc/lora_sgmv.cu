@@ -572,7 +572,9 @@ lora_status expand_unaligned_tc(const lora::ExpandArgs& a, lora_dtype dt, const 
   };
   P.stages = 2;
   while (P.stages < 4 && total(P.stages + 1) <= 225 * 1024) ++P.stages;
-  if (total(P.stages) > 225 * 1024) return LORA_OK;
+  // the rank activations of a piece are staged in the logical tile and the
+  // stages' B staging areas: at most stages + 1 slices
+  if (total(P.stages) > 225 * 1024 || a.S > P.stages + 1) return LORA_OK;
   const size_t smem = std::max<size_t>(total(P.stages), 120 * 1024);  // one CTA per SM
 
   const long slots = lora::num_piece_slots(a.tok, P.nvseg, lora::kExBM);
