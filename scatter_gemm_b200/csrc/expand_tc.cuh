@@ -203,12 +203,16 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
   };
   // base tile t into ring stage s: chunk u = j*128 + pt -> row u / kExCh,
   // logical chunk u % kExCh (two 256-byte rows per warp instruction)
+  // A producer's rows are the same for every tile (pt / kExCh + j * 128 /
+  // kExCh), so their tokens are read from shared memory once (ptok) and the
+  // copies of a tile issue back to back, none waiting on a shared-memory load.
+  int ptok[kExCh];
   auto issue_tile = [&](int t, int s) {
     int q, c0;
     tile_info(t, q, c0);
     const int cend = p.slices.off[q + 1];
     const uint32_t stage = base_ring + s * kExStageBytes;
-#pragma unroll 4
+#pragma unroll
     for (int j = 0; j < kExCh; ++j) {
       const int u = j * kExBM + pt;
       const int row = u / kExCh, c = u % kExCh;
@@ -217,7 +221,7 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
       // epilogue never stores them
       if (row < rows && col < cend)
         cp_async_16(stage + row * (kExBN * 2) + ((c ^ (row & (kExCh - 1))) << 4),
-                    p.base + static_cast<int64_t>(trow[row]) * p.ld_base + col, 16u);
+                    p.base + static_cast<int64_t>(ptok[j]) * p.ld_base + col, 16u);
     }
   };
   const int pre = min(P.base_stages, ntl);  // tiles issued before the CTA barrier
@@ -267,6 +271,8 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
     }
     cp_async_commit();
     named_bar_sync(2, kExProducers);  // trow of every row is in shared memory
+#pragma unroll
+    for (int j = 0; j < kExCh; ++j) ptok[j] = trow[(j * kExBM + pt) / kExCh];
     for (int t = 0; t < pre; ++t) {
       issue_tile(t, t);
       cp_async_commit();
@@ -395,12 +401,14 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
       if (ok) {
         constexpr int kPer = (kExBM * kExCh) / kExConsumers;
         uint4 w[kPer];
+        int tk[kPer];
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
           const int u = j * kExConsumers + ct;
           const int row = u / kExCh, c = u % kExCh;
           w[j] = *reinterpret_cast<const uint4*>(stage_p + row * (kExBN * 2) +
                                                  ((c ^ (row & (kExCh - 1))) << 4));
+          tk[j] = trow[row];
         }
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
@@ -408,8 +416,8 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
           const int row = u / kExCh, c = u % kExCh;
           const int col = c0 + 8 * c;
           if (row < rows && col < cend)
-            *reinterpret_cast<uint4*>(p.base + static_cast<int64_t>(trow[row]) * p.ld_base +
-                                      col) = w[j];
+            *reinterpret_cast<uint4*>(p.base + static_cast<int64_t>(tk[j]) * p.ld_base + col) =
+                w[j];
         }
       }
       mbar_arrive(xempty0 + 8 * s);  // the stage's shared memory may be refilled

@@ -49,6 +49,9 @@
 #ifndef LORA_EXPAND_B_STAGES
 #define LORA_EXPAND_B_STAGES 3
 #endif
+#ifndef LORA_EU_CTAS_PER_SM
+#define LORA_EU_CTAS_PER_SM 2       // element-aligned expand: CTAs per SM when they fit
+#endif
 #ifndef LORA_SHRINK_WIDE_SMEM
 #define LORA_SHRINK_WIDE_SMEM 0     // 1: one-CTA-per-SM budget when the grid fits the SMs
 #endif
@@ -562,26 +565,48 @@ lora_status expand_unaligned_tc(const lora::ExpandArgs& a, lora_dtype dt, const 
   }
   P.tiles_total = tiles;
   P.idesc = lora::make_idesc_f16(dt == LORA_BF16 ? 1 : 0, lora::kExBM, lora::kExBN);
-  P.stage_bytes = static_cast<uint32_t>(
-      round_up(lora::kEuRawBase + static_cast<int>(P.btile_bytes) + lora::kExBM * lora::kEuStageRow,
-               1024));
-  const size_t fixed = lora::kExStageBytes + static_cast<size_t>(a.S) * P.rin_bytes +
-                       4 * lora::kExBM + 1024 + 16;
+  P.srow = static_cast<uint32_t>(16 * (P.rpad / 8 + 1));
+  P.stage_bytes = static_cast<uint32_t>(round_up(
+      lora::kEuRawBase + static_cast<int>(P.btile_bytes) + lora::kExBM * static_cast<int>(P.srow),
+      1024));
+  // rank activations, row tokens, two groups' row addresses, alignment slack
+  const size_t fixed = static_cast<size_t>(a.S) * P.rin_bytes + 4 * lora::kExBM +
+                       2 * sizeof(uintptr_t) * lora::kExBM + 1024 + 16;
   auto total = [&](int nb) {
-    return static_cast<size_t>(nb) * P.stage_bytes + fixed + 8 * (3 * nb + 6);
+    return static_cast<size_t>(nb) * P.stage_bytes + fixed + 8 * (3 * nb + 7);
   };
+  // two CTAs per SM (TMEM: 2 x 256 columns) when two stages fit in half the
+  // SM's shared memory, else one CTA with up to four stages
+  const int ctas_per_sm = LORA_EU_CTAS_PER_SM >= 2 && total(2) <= 113 * 1024 ? 2 : 1;
+  const size_t cap = ctas_per_sm == 2 ? 113 * 1024 : 225 * 1024;
   P.stages = 2;
-  while (P.stages < 4 && total(P.stages + 1) <= 225 * 1024) ++P.stages;
-  // the rank activations of a piece are staged in the logical tile and the
-  // stages' B staging areas: at most stages + 1 slices
-  if (total(P.stages) > 225 * 1024 || a.S > P.stages + 1) return LORA_OK;
-  const size_t smem = std::max<size_t>(total(P.stages), 120 * 1024);  // one CTA per SM
+  while (P.stages < 4 && total(P.stages + 1) <= cap) ++P.stages;
+  // the rank activations of a piece are staged in the last stage's base area
+  // (as many slices as fit) and the B staging areas of stages stages-1 .. 0;
+  // stage 0's only when needed, since the first B tile then waits for them
+  const int nfit = lora::kEuRawBase / (lora::kExBM * static_cast<int>(P.srow));
+  if (total(P.stages) > cap || a.S > nfit + P.stages) return LORA_OK;
+  P.rin_in_stage0 = a.S > nfit + P.stages - 1 ? 1 : 0;
+  const size_t smem = std::max<size_t>(total(P.stages), kTmemCtaMinSmem);
 
   const long slots = lora::num_piece_slots(a.tok, P.nvseg, lora::kExBM);
-  const long target = dev.sms;
-  long tpc = (slots * tiles + target - 1) / target;
-  if (tpc < 1) tpc = 1;
-  if (tpc > tiles) tpc = tiles;
+  // Tiles per CTA: the split of the tiles into column groups that minimises
+  // waves x (tiles per CTA + start-up), for the pieces expected (one per 128
+  // rows plus half a piece per segment; slots beyond them find no piece and
+  // leave at once).  The start-up (tables, rank rows, first tiles) costs about
+  // two tiles' epilogues.
+  const long est = (a.tok + lora::kExBM - 1) / lora::kExBM + P.nvseg / 2;
+  const long resident = static_cast<long>(ctas_per_sm) * dev.sms;
+  long tpc = tiles, best = -1;
+  for (long t = 1; t <= tiles; ++t) {
+    const long ncg_t = (tiles + t - 1) / t;
+    const long waves = (std::max(est, 1L) * ncg_t + resident - 1) / resident;
+    const long cost = waves * ((tiles + ncg_t - 1) / ncg_t + 2);
+    if (best < 0 || cost < best) {
+      best = cost;
+      tpc = t;
+    }
+  }
   P.tiles_per_cta = static_cast<int>(tpc);
   const long ncg = (tiles + tpc - 1) / tpc;
   if (slots * ncg >= (1L << 31)) return LORA_OK;

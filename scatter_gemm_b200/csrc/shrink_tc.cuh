@@ -247,37 +247,45 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
         if (!rowok[h]) continue;
         const uintptr_t a = reinterpret_cast<uintptr_t>(rowp[h] + k0);
         const uintptr_t a0 = a & ~static_cast<uintptr_t>(15);
-        const uintptr_t a1 = (a + 2 * nv + 15) & ~static_cast<uintptr_t>(15);
-        for (uintptr_t b = a0; b < a1; b += 16)
-          cp_async_16_ca(st + rawo[h] + static_cast<uint32_t>(b - a0),
-                         reinterpret_cast<const void*>(b));
+        // blocks holding at least one of the nv elements (<= 9)
+        const int nb = static_cast<int>(((a + 2 * nv + 15) & ~static_cast<uintptr_t>(15)) - a0) >> 4;
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(a0);
+#pragma unroll
+        for (int b = 0; b < 9; ++b)
+          if (b < nb) cp_async_16_ca(st + rawo[h] + 16 * b, src + 16 * b);
       }
     };
+    // The staged row is a byte stream: element k0 + e sits at byte off + 2e
+    // (off = source address & 15).  Word k of the shifted row (elements
+    // 2k, 2k+1) is the 4 bytes at off + 4k: staged words q + k and q + k + 1
+    // (q = off / 4) funnel-shifted by 16 bits when off % 4 == 2.  The word
+    // index is an address offset, so every load below has a constant offset
+    // from the row's base; elements past K are zeroed in the last stage only.
     auto realign_rows = [&](int j) {
-      const uint32_t st = sbase + (j % P.stages) * P.stage_bytes;
-      const uint8_t* stp = smem + (j % P.stages) * P.stage_bytes;
+      uint8_t* stp = smem + (j % P.stages) * P.stage_bytes;
       const int k0 = LORA_KB(j) * kTcBK;
       const int nv = min(kTcAtomK, p.K - k0);
 #pragma unroll
       for (int h = 0; h < 3; ++h) {
         if (!rowok[h]) continue;
         const int off = static_cast<int>(reinterpret_cast<uintptr_t>(rowp[h] + k0) & 15);
-        const uint4* raw = reinterpret_cast<const uint4*>(stp + rawo[h]);
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(stp + rawo[h]) + (off >> 2);
+        const uint32_t fs = (off & 2) * 8;  // 0 or 16 bits
+        uint8_t* dst = stp + dsto[h];
+        const int sw = rown[h] & 7;
+        uint32_t ws[33];  // every staged word first: the stores below may alias them
+#pragma unroll
+        for (int i = 0; i < 33; ++i) ws[i] = w[i];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          const int keep = min(8, max(0, nv - 8 * c));
-          uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (keep > 0) {
-            const int pos = off + 16 * c, blk = pos >> 4, sh = pos & 15;
-            const uint4 w0 = raw[blk];
-            const uint4 w1 = (sh != 0 && blk < 8) ? raw[blk + 1] : make_uint4(0u, 0u, 0u, 0u);
-            v = keep_elems(bytes_at(w0, w1, sh), keep);
-          }
-          *reinterpret_cast<uint4*>(const_cast<uint8_t*>(stp) + dsto[h] +
-                                    ((c ^ (rown[h] & 7)) << 4)) = v;
+          uint32_t o[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) o[i] = __funnelshift_r(ws[4 * c + i], ws[4 * c + i + 1], fs);
+          uint4 v = make_uint4(o[0], o[1], o[2], o[3]);
+          if (nv < kTcAtomK) v = keep_elems(v, nv - 8 * c);
+          *reinterpret_cast<uint4*>(dst + ((c ^ sw) << 4)) = v;
         }
       }
-      (void)st;
     };
     const int lag = P.stages - 1;
     for (int i = 0; i < nk && ok; ++i) {

@@ -49,6 +49,18 @@ def test_expand_element_aligned_ranks(r, rs):
     assert lora.last_path() & T
 
 
+@pytest.mark.parametrize("slices", [[300, 41], [64, 64, 64, 64]])
+def test_expand_element_aligned_rank64_slice_counts(slices):
+    # rank 64: one slice's staged rank rows fill the last stage's base area, the
+    # others go to the B staging areas (two slices) or also stage 0's (S > 3 is
+    # refused by the tensor path and runs on the CUDA cores)
+    p = make_problem("qkv", seed=65, tok=200, K=64, slices=slices, r=64, rs=64,
+                     misalign=1, ld_pad=3, col_lead=1)
+    check_expand(p)
+    if len(slices) <= 3:
+        assert lora.last_path() & T
+
+
 def test_expand_element_aligned_grouped_zero_scaling_and_lead_trail():
     p = make_problem("many_small", seed=70, tok=900, nseg=120, K=64, slices=[250, 70, 70],
                      misalign=3, lead=9, trail=4, col_lead=5)
