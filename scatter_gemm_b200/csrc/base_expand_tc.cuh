@@ -300,15 +300,28 @@ base_expand_tc_kernel(const __grid_constant__ BaseExpandTcParams P) {
     tc_fence_before();
     named_bar_sync(1, kTcBM);  // the whole tile is staged
     if (ok) {
-      // coalesced write-back: chunk u = j*128 + tid -> row u / 16, chunk u % 16
-#pragma unroll 4
-      for (int j = 0; j < (kTcBM * 16) / kTcBM; ++j) {
-        const int u = j * kTcBM + tid;
-        const int row = u / 16, c = u % 16;
-        const int col = c0 + 8 * c;
-        if (row < rows && col < cend)
-          *reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(trow[row]) * p.ld_out + col) =
-              *reinterpret_cast<const uint4*>(stile + row * (kBeBN * 2) + ((c ^ (row & 15)) << 4));
+      // coalesced write-back: chunk u = j*128 + tid -> row u / 16, chunk u % 16;
+      // four chunks at a time, their shared-memory reads before the stores
+      constexpr int kBatch = 4;
+#pragma unroll
+      for (int j0 = 0; j0 < 16; j0 += kBatch) {
+        uint4 w[kBatch];
+        int tk[kBatch];
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+          const int u = (j0 + k) * kTcBM + tid;
+          const int row = u / 16, c = u % 16;
+          w[k] = *reinterpret_cast<const uint4*>(stile + row * (kBeBN * 2) + ((c ^ (row & 15)) << 4));
+          tk[k] = trow[row];
+        }
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+          const int u = (j0 + k) * kTcBM + tid;
+          const int row = u / 16, c = u % 16;
+          const int col = c0 + 8 * c;
+          if (row < rows && col < cend)
+            *reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(tk[k]) * p.ld_out + col) = w[k];
+        }
       }
     }
   }

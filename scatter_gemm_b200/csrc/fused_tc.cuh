@@ -198,13 +198,17 @@ fused_tc_kernel(const __grid_constant__ FusedTcParams P) {
       if (k < pe.S && g >= P.tile_prefix[k]) q = k;
     c0 = pe.slices.off[q] + (g - P.tile_prefix[q]) * kExBN;
   };
-  // base tile t into ring stage s: chunk u = j*128 + pt -> row u / kExCh, chunk u % kExCh
+  // base tile t into ring stage s: chunk u = j*128 + pt -> row u / kExCh, chunk
+  // u % kExCh.  A producer's rows are the same for every tile, so their tokens
+  // sit in registers (ptok, filled once trow is complete) and the copies of a
+  // tile issue back to back, none waiting on a shared-memory load.
+  int ptok[kExCh];
   auto issue_tile = [&](int t, int s) {
     int q, c0;
     tile_cols(t, q, c0);
     const int cend = pe.slices.off[q + 1];
     const uint32_t stage = xstage(s);
-#pragma unroll 4
+#pragma unroll
     for (int j = 0; j < kExCh; ++j) {
       const int u = j * kExBM + pt;
       const int row = u / kExCh, c = u % kExCh;
@@ -213,7 +217,7 @@ fused_tc_kernel(const __grid_constant__ FusedTcParams P) {
       // epilogue never stores them
       if (row < rows && col < cend)
         cp_async_16(stage + row * (kExBN * 2) + ((c ^ (row & (kExCh - 1))) << 4),
-                    pe.base + static_cast<int64_t>(trow[row]) * pe.ld_base + col, 16u);
+                    pe.base + static_cast<int64_t>(ptok[j]) * pe.ld_base + col, 16u);
     }
   };
   auto load_b = [&](int t, int sp) {
@@ -240,6 +244,8 @@ fused_tc_kernel(const __grid_constant__ FusedTcParams P) {
     const uint16_t* xr[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) xr[j] = ps.x + static_cast<int64_t>(trow[rr + 16 * j]) * ps.ld_x;
+#pragma unroll
+    for (int j = 0; j < kExCh; ++j) ptok[j] = trow[(j * kExBM + pt) / kExCh];
     const int lag = P.stages - 1;
     for (int i = 0; i < nk && ok; ++i) {
       const int s = i % P.stages;
@@ -480,18 +486,32 @@ fused_tc_kernel(const __grid_constant__ FusedTcParams P) {
       named_bar_sync(1 + grp, kFuGroup);  // every row of the tile is updated
       // (b) coalesced write-back of the rows of the piece: chunk u = j*128 + gt
       const int cend = pe.slices.off[q + 1];
+      //     four chunks at a time: their shared-memory reads first, then the
+      //     stores (a load may not pass a store through a generic pointer)
       if (ok) {
         constexpr int kPer = (kExBM * kExCh) / kFuGroup;
-#pragma unroll 4
-        for (int j = 0; j < kPer; ++j) {
-          const int u = j * kFuGroup + gt;
-          const int row = u / kExCh, c = u % kExCh;
-          const int col = c0 + 8 * c;
-          if (row < rows && col < cend)
-            *reinterpret_cast<uint4*>(pe.base + static_cast<int64_t>(trow[row]) * pe.ld_base +
-                                      col) =
-                *reinterpret_cast<const uint4*>(stage_p + row * (kExBN * 2) +
-                                                ((c ^ (row & (kExCh - 1))) << 4));
+        constexpr int kBatch = 4;
+#pragma unroll
+        for (int j0 = 0; j0 < kPer; j0 += kBatch) {
+          uint4 w[kBatch];
+          int tk[kBatch];
+#pragma unroll
+          for (int k = 0; k < kBatch; ++k) {
+            const int u = (j0 + k) * kFuGroup + gt;
+            const int row = u / kExCh, c = u % kExCh;
+            w[k] = *reinterpret_cast<const uint4*>(stage_p + row * (kExBN * 2) +
+                                                   ((c ^ (row & (kExCh - 1))) << 4));
+            tk[k] = trow[row];
+          }
+#pragma unroll
+          for (int k = 0; k < kBatch; ++k) {
+            const int u = (j0 + k) * kFuGroup + gt;
+            const int row = u / kExCh, c = u % kExCh;
+            const int col = c0 + 8 * c;
+            if (row < rows && col < cend)
+              *reinterpret_cast<uint4*>(pe.base + static_cast<int64_t>(tk[k]) * pe.ld_base + col) =
+                  w[k];
+          }
         }
       }
       mbar_arrive(xempty0 + 8 * s);
