@@ -491,14 +491,27 @@ lora_status expand_tc(const lora::ExpandArgs& a, lora_dtype dt, const Grouping& 
 
   // shared memory: base ring, rank activations, B ring, row tables, barriers
   P.b_stages = LORA_EXPAND_B_STAGES;
-  const size_t fixed = static_cast<size_t>(a.S) * P.rin_bytes +
-                       static_cast<size_t>(P.b_stages) * P.btile_bytes + 1024 + 512 + 16;
   auto total = [&](int bs) {
+    const size_t fixed = static_cast<size_t>(a.S) * P.rin_bytes +
+                         static_cast<size_t>(P.b_stages) * P.btile_bytes + 1024 + 512 + 16;
     return ((static_cast<size_t>(bs) * lora::kExStageBytes + 1023) & ~size_t(1023)) + fixed +
            8 * (2 * P.b_stages + 5 + 2 * bs);
   };
-  // two CTAs per SM only when both accumulators fit twice in TMEM (512 columns)
-  const int ctas_per_sm = (LORA_EXPAND_CTAS_PER_SM >= 2 && lora::kExTmemCols <= 256) ? 2 : 1;
+  // two CTAs per SM when both accumulators fit twice in TMEM (512 columns) and
+  // two base stages fit in half the shared memory, with a B ring of two if
+  // three do not fit; otherwise one CTA per SM with a deeper base ring.  (The
+  // grid is sized for two CTAs per SM either way: sized for one, the rank-64
+  // gate_up expand measured 188 us against 140 us.)
+  const int grid_ctas_per_sm =
+      (LORA_EXPAND_CTAS_PER_SM >= 2 && lora::kExTmemCols <= 256) ? 2 : 1;
+  int ctas_per_sm = grid_ctas_per_sm;
+  if (ctas_per_sm == 2 && total(2) > 113 * 1024) {
+    P.b_stages = 2;
+    if (total(2) > 113 * 1024) {
+      P.b_stages = LORA_EXPAND_B_STAGES;
+      ctas_per_sm = 1;
+    }
+  }
   const size_t cap = (ctas_per_sm >= 2 ? 113 : 225) * 1024;
   P.base_stages = 2;
   while (P.base_stages < 7 && total(P.base_stages + 1) <= cap) ++P.base_stages;
@@ -514,7 +527,7 @@ lora_status expand_tc(const lora::ExpandArgs& a, lora_dtype dt, const Grouping& 
     return LORA_ERR_CUDA;
 
   const long slots = lora::num_piece_slots(a.tok, P.nvseg, lora::kExBM);
-  const long target = static_cast<long>(ctas_per_sm) * dev.sms * LORA_EXPAND_WAVES;
+  const long target = static_cast<long>(grid_ctas_per_sm) * dev.sms * LORA_EXPAND_WAVES;
   long tpc = (slots * tiles + target - 1) / target;
   if (tpc < 1) tpc = 1;
   if (tpc > tiles) tpc = tiles;
