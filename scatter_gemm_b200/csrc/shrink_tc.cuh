@@ -215,7 +215,7 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
   if (!AL && warp < 4) {
     // =========================== producer, element-aligned rows
     // Thread m stages x row m and A rows m and m + 128 of the stage's 64 K
-    // columns: copy the covering 16-byte blocks (cp.async through L1, one row
+    // columns: copy the covering 16-byte blocks (16-byte cp.async, one row
     // per thread), and once they have landed (lagged like the aligned path)
     // shift them into the swizzled K-major layout, zero past K.
     const int m = tid;
@@ -252,7 +252,7 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
         const uint8_t* src = reinterpret_cast<const uint8_t*>(a0);
 #pragma unroll
         for (int b = 0; b < 9; ++b)
-          if (b < nb) cp_async_16_ca(st + rawo[h] + 16 * b, src + 16 * b);
+          if (b < nb) cp_async_16(st + rawo[h] + 16 * b, src + 16 * b, 16u);
       }
     };
     // The staged row is a byte stream: element k0 + e sits at byte off + 2e
