@@ -23,18 +23,44 @@ namespace lora {
 
 constexpr int kGroupThreads = 1024;
 constexpr int kGroupMaxAdapters = 8192;
+// Shared-memory bound (bytes) for staging seg_indptr and the segment bases
+// next to the adapter counts; larger tables are read from global memory.
+constexpr int kGroupStageBytes = 46 * 1024;  // under the 48 KB default with the static part
+
+__host__ __device__ __forceinline__ bool group_stages_tables(int nseg, int L) {
+  return 4ll * (static_cast<long long>(L) + 2ll * nseg + 1) <= kGroupStageBytes;
+}
+
+// Entries of a[0..n) that are <= v (a sorted), in shared memory.
+__device__ __forceinline__ int count_le_smem(const int* a, int n, int v) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (a[mid] <= v) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
 
 __global__ void __launch_bounds__(kGroupThreads)
 group_rows_kernel(const int32_t* __restrict__ seg_indptr, const int32_t* __restrict__ weight_indices,
                   int nseg, int L, int tok, int32_t* __restrict__ vseg_indptr,
                   int32_t* __restrict__ seg_base, int32_t* __restrict__ row_list) {
-  extern __shared__ int cnt[];  // [L] counts, then cursors
+  // [L] counts, then cursors; when the tables fit (group_stages_tables):
+  // [nseg + 1] clamped seg_indptr and [nseg] segment bases, so that the row
+  // pass below searches shared memory instead of chasing global loads
+  extern __shared__ int cnt[];
   __shared__ int warp_tot[32];
   const int tid = threadIdx.x;
+  const bool staged = group_stages_tables(nseg, L);
+  int* sidx = cnt + L;
+  int* sbase = sidx + nseg + 1;
   for (int a = tid; a < L; a += blockDim.x) cnt[a] = 0;
+  if (staged)
+    for (int i = tid; i <= nseg; i += blockDim.x) sidx[i] = clampi(seg_indptr[i], 0, tok);
   __syncthreads();
+  auto bound = [&](int i) { return staged ? sidx[i] : clampi(seg_indptr[i], 0, tok); };
   for (int s = tid; s < nseg; s += blockDim.x) {
-    const int lo = clampi(seg_indptr[s], 0, tok), hi = clampi(seg_indptr[s + 1], 0, tok);
+    const int lo = bound(s), hi = bound(s + 1);
     if (hi > lo) atomicAdd(&cnt[clampi(weight_indices[s], 0, L - 1)], hi - lo);
   }
   __syncthreads();
@@ -75,16 +101,17 @@ group_rows_kernel(const int32_t* __restrict__ seg_indptr, const int32_t* __restr
   __syncthreads();
 
   for (int s = tid; s < nseg; s += blockDim.x) {
-    const int lo = clampi(seg_indptr[s], 0, tok), hi = clampi(seg_indptr[s + 1], 0, tok);
-    seg_base[s] = hi > lo ? atomicAdd(&cnt[clampi(weight_indices[s], 0, L - 1)], hi - lo) : 0;
+    const int lo = bound(s), hi = bound(s + 1);
+    const int b = hi > lo ? atomicAdd(&cnt[clampi(weight_indices[s], 0, L - 1)], hi - lo) : 0;
+    if (staged) sbase[s] = b; else seg_base[s] = b;
   }
   __syncthreads();
 
-  const int rlo = clampi(seg_indptr[0], 0, tok), rhi = clampi(seg_indptr[nseg], 0, tok);
+  const int rlo = bound(0), rhi = bound(nseg);
   for (int i = rlo + tid; i < rhi; i += blockDim.x) {
-    const int s = count_le(seg_indptr, nseg + 1, i) - 1;
+    const int s = (staged ? count_le_smem(sidx, nseg + 1, i) : count_le(seg_indptr, nseg + 1, i)) - 1;
     if (s < 0 || s >= nseg) continue;
-    const int g = seg_base[s] + (i - clampi(seg_indptr[s], 0, tok));
+    const int g = (staged ? sbase[s] : seg_base[s]) + (i - bound(s));
     if (g >= 0 && g < tok) row_list[g] = i;
   }
 }

@@ -293,7 +293,10 @@ lora_status maybe_group(const int32_t* seg_indptr, const int32_t* weight_indices
   int32_t* vseg = w;
   int32_t* seg_base = vseg + a16(static_cast<size_t>(L) + 1);
   int32_t* rows = seg_base + a16(static_cast<size_t>(nseg));
-  lora::group_rows_kernel<<<1, lora::kGroupThreads, sizeof(int) * L, st>>>(
+  const size_t gsmem = sizeof(int) * (lora::group_stages_tables(nseg, L)
+                                          ? static_cast<size_t>(L) + 2 * static_cast<size_t>(nseg) + 1
+                                          : static_cast<size_t>(L));
+  lora::group_rows_kernel<<<1, lora::kGroupThreads, gsmem, st>>>(
       seg_indptr, weight_indices, nseg, L, tok, vseg, seg_base, rows);
   ++g_launches;
   if (launch_status() != LORA_OK) return LORA_ERR_CUDA;
