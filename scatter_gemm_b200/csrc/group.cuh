@@ -23,9 +23,10 @@ namespace lora {
 
 constexpr int kGroupThreads = 1024;
 constexpr int kGroupMaxAdapters = 8192;
-// Shared-memory bound (bytes) for staging seg_indptr and the segment bases
-// next to the adapter counts; larger tables are read from global memory.
-constexpr int kGroupStageBytes = 46 * 1024;  // under the 48 KB default with the static part
+// Shared-memory bound (bytes, the kernel's dynamic limit) for staging
+// seg_indptr and the segment bases next to the adapter counts (up to about
+// 25,000 segments); larger tables are read from global memory.
+constexpr int kGroupStageBytes = 200 * 1024;
 
 __host__ __device__ __forceinline__ bool group_stages_tables(int nseg, int L) {
   return 4ll * (static_cast<long long>(L) + 2ll * nseg + 1) <= kGroupStageBytes;

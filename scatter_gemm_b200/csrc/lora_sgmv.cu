@@ -135,6 +135,8 @@ const DeviceFacts* device_facts() {
     f.sms = sms;
     set_kernel_attrs<lora::Bf16>();
     set_kernel_attrs<lora::Fp16>();
+    cudaFuncSetAttribute(lora::group_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         lora::kGroupStageBytes);
     // can 16 CTAs of the shrink (at its largest two-per-SM footprint) form a cluster?
     cudaLaunchConfig_t cfg{};
     cudaLaunchAttribute attr[1];
@@ -288,6 +290,7 @@ lora_status maybe_group(const int32_t* seg_indptr, const int32_t* weight_indices
                         Grouping& g) {
   g = Grouping{};
   if (!ws || nseg <= L || L > lora::kGroupMaxAdapters) return LORA_OK;
+  if (!device_facts()) return LORA_ERR_CUDA;  // sets the pass's shared-memory limit
   if (!aligned_to(ws, 16) || ws_bytes < workspace_ints(tok, nseg, L) * 4) return LORA_OK;
   int32_t* w = static_cast<int32_t*>(ws);
   int32_t* vseg = w;
