@@ -532,11 +532,24 @@ lora_status expand_tc(const lora::ExpandArgs& a, lora_dtype dt, const Grouping& 
                  static_cast<uint64_t>(a.rs) * 2, P.rpad, lora::kExBN, swz))
     return LORA_ERR_CUDA;
 
+  // Tiles per CTA: the split of the tiles into column groups that minimises
+  // waves x (tiles per CTA + start-up) with every slot counted as a piece (the
+  // start-up costs about two tiles' epilogues).  It keeps the grid within one
+  // wave where the plain quotient would spill a few CTAs into a second (qkv at
+  // tok 16384: 23 tiles per CTA gave three column groups and 408 CTAs for 296
+  // places).
   const long slots = lora::num_piece_slots(a.tok, P.nvseg, lora::kExBM);
-  const long target = static_cast<long>(grid_ctas_per_sm) * dev.sms * LORA_EXPAND_WAVES;
-  long tpc = (slots * tiles + target - 1) / target;
-  if (tpc < 1) tpc = 1;
-  if (tpc > tiles) tpc = tiles;
+  const long resident = static_cast<long>(grid_ctas_per_sm) * dev.sms * LORA_EXPAND_WAVES;
+  long tpc = tiles, best = -1;
+  for (long t = 1; t <= tiles; ++t) {
+    const long ncg_t = (tiles + t - 1) / t;
+    const long waves = (slots * ncg_t + resident - 1) / resident;
+    const long cost = waves * ((tiles + ncg_t - 1) / ncg_t + 2);
+    if (best < 0 || cost < best) {
+      best = cost;
+      tpc = t;
+    }
+  }
   P.tiles_per_cta = static_cast<int>(tpc);
   const long ncg = (tiles + tpc - 1) / tpc;
   if (slots * ncg >= (1L << 31)) return LORA_ERR_UNSUPPORTED;
