@@ -137,6 +137,8 @@ const DeviceFacts* device_facts() {
     set_kernel_attrs<lora::Fp16>();
     cudaFuncSetAttribute(lora::group_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          lora::kGroupStageBytes);
+    cudaFuncSetAttribute(lora::group_rows_small_kernel,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, lora::kGroupStageBytes);
     // can 16 CTAs of the shrink (at its largest two-per-SM footprint) form a cluster?
     cudaLaunchConfig_t cfg{};
     cudaLaunchAttribute attr[1];
@@ -296,11 +298,17 @@ lora_status maybe_group(const int32_t* seg_indptr, const int32_t* weight_indices
   int32_t* vseg = w;
   int32_t* seg_base = vseg + a16(static_cast<size_t>(L) + 1);
   int32_t* rows = seg_base + a16(static_cast<size_t>(nseg));
-  const size_t gsmem = sizeof(int) * (lora::group_stages_tables(nseg, L)
-                                          ? static_cast<size_t>(L) + 2 * static_cast<size_t>(nseg) + 1
-                                          : static_cast<size_t>(L));
-  lora::group_rows_kernel<<<1, lora::kGroupThreads, gsmem, st>>>(
-      seg_indptr, weight_indices, nseg, L, tok, vseg, seg_base, rows);
+  if (lora::group_small_fits(nseg, L, tok)) {
+    lora::group_rows_small_kernel<<<1, lora::kGroupThreads,
+                                    static_cast<size_t>(lora::group_small_smem(nseg, L, tok)), st>>>(
+        seg_indptr, weight_indices, nseg, L, tok, vseg, rows);
+  } else {
+    const size_t gsmem = sizeof(int) * (lora::group_stages_tables(nseg, L)
+                                            ? static_cast<size_t>(L) + 3 * static_cast<size_t>(nseg) + 1
+                                            : static_cast<size_t>(L));
+    lora::group_rows_kernel<<<1, lora::kGroupThreads, gsmem, st>>>(
+        seg_indptr, weight_indices, nseg, L, tok, vseg, seg_base, rows);
+  }
   ++g_launches;
   if (launch_status() != LORA_OK) return LORA_ERR_CUDA;
   g.vseg_indptr = vseg;
