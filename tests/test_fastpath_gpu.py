@@ -107,6 +107,20 @@ def test_many_segments_with_workspace_are_grouped():
     assert not lora.last_path() & G
 
 
+@pytest.mark.parametrize("L,nseg,tok", [(8, 20, 2000), (300, 400, 1200)])
+def test_grouping_long_segments_and_many_adapters(L, nseg, tok):
+    # random segment lengths (many longer than 64 rows, listed by whole warps)
+    # with repeated adapters; and more adapters than the per-warp counters
+    # hold (the grouping pass with shared counters)
+    p = make_problem("qkv", seed=24 + L, tok=tok, K=192, slices=[128, 64, 64], L=L, nseg=nseg,
+                     recipe="random", lead=3, trail=2)
+    assert int((np.diff(p.seg_indptr) > 64).sum()) > 0 or L > 256
+    check_shrink(p, workspace=True)
+    assert lora.last_path() & G and lora.last_path() & T
+    check_expand(p, workspace=True)
+    assert lora.last_path() & G and lora.last_path() & T
+
+
 def test_small_token_counts_split_k_over_a_cluster():
     p = make_problem("qkv", seed=23, tok=50, K=4096)
     check_shrink(p)
