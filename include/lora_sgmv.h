@@ -18,9 +18,11 @@
  *    tensor of a call except `scalings`, which is fp32.  Accumulation is fp32;
  *    each output element is rounded once, to nearest even.
  *  - All tensors are row-major with an explicit leading dimension (in
- *    elements).  Any element-aligned pointer is accepted; faster kernels are
- *    picked at run time when pointers and leading dimensions are 16-byte
- *    aligned.
+ *    elements).  Any element-aligned pointer is accepted.  The tensor-core
+ *    kernels take rows at any 2-byte offset: 16-byte-aligned rows go straight
+ *    into their stages, others are staged as the 16-byte blocks that cover
+ *    them and shifted into place.  CUDA-core kernels remain for ranks above
+ *    64 and, in the shrink, S*rs above 256.
  *  - Tables (int32, in device memory):
  *      seg_indptr[nseg+1]   segment s covers sorted rows [seg_indptr[s], seg_indptr[s+1]);
  *                           non-decreasing, inside [0, tok]; empty segments allowed;
@@ -95,8 +97,8 @@ enum {
 
 /* Kernel path bits reported by lora_last_path. */
 enum {
-  LORA_PATH_GENERAL = 1, /* element-aligned CUDA-core kernel                       */
-  LORA_PATH_TENSOR = 2,  /* tcgen05 tensor-core kernel (16-byte-aligned inputs)     */
+  LORA_PATH_GENERAL = 1, /* CUDA-core kernel (r > 64; shrink S*rs > 256)           */
+  LORA_PATH_TENSOR = 2,  /* tcgen05 tensor-core kernel (any element alignment)      */
   LORA_PATH_GROUPED = 4, /* rows grouped by adapter first (workspace, many segments) */
   LORA_PATH_SPLITK = 8,  /* shrink K range split over a thread-block cluster        */
   LORA_PATH_FUSED = 16   /* lora_shrink_expand ran both ops in one launch            */

@@ -1,9 +1,9 @@
-// general.cuh -- element-aligned CUDA-core kernels of the shrink and expand.
+// general.cuh -- CUDA-core kernels of the shrink and expand.
 //
 // These accept any pointer alignment, leading dimension, rank, K and slice
-// layout (2-byte accesses only), so they are the path for inputs that the
-// 16-byte-aligned tensor-core kernels cannot take (e.g. a 4-byte pointer
-// offset with K = 3583).  Both use the on-device piece scheduler of sched.cuh.
+// layout (2-byte accesses only), so they are the path for shapes the
+// tensor-core kernels do not take: ranks above 64, a padded shrink width
+// S*rs above 256.  Both use the on-device piece scheduler of sched.cuh.
 #pragma once
 
 #include "common.cuh"

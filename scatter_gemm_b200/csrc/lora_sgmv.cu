@@ -5,10 +5,12 @@
 // synchronised: every call enqueues its kernels on the caller's stream.
 //
 // Kernel selection (run time, from pointers and sizes only):
-//   tensor-core kernels (shrink_tc / expand_tc) when every tensor they stream
-//   is 16-byte aligned with 16-byte-multiple row strides, K % 8 == 0, the
-//   padded shrink width S*rs <= 256, slice starts % 8 == 0 and r <= 64 for the
-//   expand; otherwise the element-aligned CUDA-core kernels of general.cuh.
+//   shrink: shrink_tc when the padded width S*rs <= 256, its aligned variant
+//   when x and A rows are 16-byte aligned with K % 8 == 0 (else the variant
+//   that stages and shifts element-aligned rows); expand: expand_tc when every
+//   tensor it streams is 16-byte aligned with 16-byte-multiple row strides,
+//   slice starts % 8 == 0 and r <= 64, else expand_unaligned for r <= 64; the
+//   CUDA-core kernels of general.cuh for what remains (r > 64, S*rs > 256).
 //   With a workspace and more segments than adapters the tensor-core kernels
 //   run on the adapter-grouped schedule of group.cuh.
 #include <cuda.h>

@@ -1,4 +1,5 @@
-// shrink_tc.cuh -- tensor-core shrink for 16-byte-aligned inputs (sm_100a).
+// shrink_tc.cuh -- tensor-core shrink (sm_100a); rows at any 2-byte offset in
+// the element-aligned variant (AL = false, below).
 //
 // One CTA computes one piece (<= 128 sorted rows of one segment, from the
 // scheduler of sched.cuh) times one K range:
