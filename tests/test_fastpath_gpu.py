@@ -107,12 +107,14 @@ def test_many_segments_with_workspace_are_grouped():
     assert not lora.last_path() & G
 
 
-@pytest.mark.parametrize("L,nseg,tok", [(8, 20, 2000), (300, 400, 1200)])
-def test_grouping_long_segments_and_many_adapters(L, nseg, tok):
-    # random segment lengths (many longer than 64 rows, listed by whole warps)
-    # with repeated adapters; and more adapters than the per-warp counters
-    # hold (the grouping pass with shared counters)
-    p = make_problem("qkv", seed=24 + L, tok=tok, K=192, slices=[128, 64, 64], L=L, nseg=nseg,
+@pytest.mark.parametrize("L,nseg,tok,K", [(8, 20, 2000, 192), (300, 400, 1200, 192),
+                                           (16, 2100, 30000, 64)])
+def test_grouping_long_segments_and_many_adapters(L, nseg, tok, K):
+    # random segment lengths with repeated adapters: few segments (the pass
+    # with block-wide counters); more adapters than the per-warp counters hold;
+    # and over 2,048 segments (the per-warp pass), some longer than 64 rows
+    # (listed by whole warps)
+    p = make_problem("qkv", seed=24 + L, tok=tok, K=K, slices=[128, 64, 64], L=L, nseg=nseg,
                      recipe="random", lead=3, trail=2)
     assert int((np.diff(p.seg_indptr) > 64).sum()) > 0 or L > 256
     check_shrink(p, workspace=True)
