@@ -405,7 +405,7 @@ lora_status shrink_tc(const lora::ShrinkArgs& a, lora_dtype dt, const Grouping& 
   const size_t recv_full = cs > 1 ? static_cast<size_t>(lora::kTcBM) * P.npad * 4 : 0;
   auto smem_for = [&](int stages, size_t recv) {
     return static_cast<size_t>(stages) * P.stage_bytes + recv + 1024 + 8 * (2 * stages + 3) +
-           8 * lora::kTcBM;
+           8 * lora::kTcBM + 8 * 16;  // row indices, ready barriers
   };
   auto stages_for = [&](size_t recv) {
     int st = 2;
@@ -413,7 +413,7 @@ lora_status shrink_tc(const lora::ShrinkArgs& a, lora_dtype dt, const Grouping& 
     return st;
   };
   // a separate receive buffer when it leaves at least three stages; otherwise
-  // the partials are received in the ring after a cluster barrier
+  // the partials are received in the ring, each CTA's once its MMAs are done
   P.stages = stages_for(recv_full);
   P.recv_in_ring = 0;
   if (cs > 1 && P.stages < 3) {

@@ -115,6 +115,9 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
   const uint32_t recv_bar = done_bar + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * P.stages + 2);
   int64_t* xrow_tok = reinterpret_cast<int64_t*>(bars + 2 * P.stages + 3);  // [128] x row index
+  // receive buffer in the ring: ready[c] completes once CTA c of the cluster
+  // has finished its MMAs (its ring may then receive partials)
+  const uint32_t ready0 = smem_u32(xrow_tok + kTcBM);  // [csplit] mbarriers
 
   // barriers and TMEM first, so that their latency overlaps the table reads
   if (tid == 0) {
@@ -124,6 +127,8 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
     }
     mbar_init(done_bar, 1);
     mbar_init(recv_bar, 1);
+    if (P.recv_in_ring)
+      for (int c = 0; c < P.csplit; ++c) mbar_init(ready0 + 8 * c, 1);
     fence_mbar_init();
     if (AL) tma_prefetch_desc(&P.tmap_A);
   }
@@ -131,10 +136,9 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
     tmem_alloc(smem_u32(tmem_slot), P.tmem_cols);
     tmem_relinquish();
   }
-  // the receive barrier must be initialised before any peer pushes into it:
-  // arrive now, wait just before the first push (a receive buffer in the ring
-  // has a cluster barrier of its own after the MMAs instead)
-  const bool early_arrive = P.csplit > 1 && !P.recv_in_ring;
+  // the receive barrier (and the ready barriers) must be initialised before
+  // any peer pushes or arrives: arrive now, wait after the MMAs
+  const bool early_arrive = P.csplit > 1;
   if (early_arrive) cluster_arrive_relaxed();
 
   // ---- piece of this cluster (identical in all its CTAs).  Rows of a block
@@ -441,16 +445,23 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
     ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
   }
   if (P.csplit > 1) {
-    if (early_arrive) cluster_wait();  // every receive barrier of the cluster is initialised
-    else cluster_sync();  // every CTA's MMAs are done: its ring may receive partials
+    cluster_wait();  // every receive and ready barrier of the cluster is initialised
+    // a receive buffer in the ring: this CTA's MMAs are done, so tell every
+    // CTA of the cluster that its pushes may come (release: the MMAs' reads
+    // of the ring come first)
+    if (P.recv_in_ring && tid < P.csplit) mbar_arrive_cluster(mapa_shared(ready0 + 8 * split, tid));
   }
   if (warp < 4) {
     tc_fence_after();
     const int m = tid;
     const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     // split-K: row m goes to CTA m / R of the cluster, into the slot of this
-    // CTA's rank
+    // CTA's rank; into a ring, only once that CTA is ready (its MMAs done)
     const int owner = m / R;
+    if (P.recv_in_ring) {
+      if (ok) ok = mbar_wait_cluster(ready0 + 8 * owner, 0);
+      ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+    }
     const uint32_t rdst = P.csplit > 1
         ? mapa_shared(smem_u32(recv) + 4u * static_cast<uint32_t>((split * R + m % R) * P.npad),
                       owner)
