@@ -63,6 +63,8 @@ static_assert(kExBN == 64 || kExBN == 128 || kExBN == 256, "expand tile width");
 
 struct ExpandTcParams {
   CUtensorMap tmap_B;  // 2-D [L*N_tot rows, r cols] (row stride rs), box {rpad, 128}
+  CUtensorMap tmap_R;  // 3-D [tok rows, S slices, r cols] of in_r, box {rpad, 1, 128}
+  int rin_tma;         // the rank activations by TMA (sorted rows contiguous: no grouping)
   ExpandArgs a;
   const int32_t* row_list;     // grouped schedule (or null)
   const int32_t* vseg_indptr;  // grouped schedule (or null)
@@ -139,6 +141,7 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
       mbar_init(bfull0 + 8 * s, 1);
       mbar_init(bempty0 + 8 * s, 1);
     }
+    mbar_init(rin_bar, P.rin_tma ? 1 : kExProducers);
     fence_mbar_init();
   }
   if (tid == 32) {
@@ -146,7 +149,6 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
       mbar_init(tfull0 + 8 * b, 1);
       mbar_init(tempty0 + 8 * b, kExConsumers);
     }
-    mbar_init(rin_bar, kExProducers);
     for (int s = 0; s < P.base_stages; ++s) {
       mbar_init(xfull0 + 8 * s, kExProducers);
       mbar_init(xempty0 + 8 * s, kExConsumers);
@@ -154,7 +156,10 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
     fence_mbar_init();
   }
   if (warp == 0) {
-    if (lane == 0) tma_prefetch_desc(&P.tmap_B);
+    if (lane == 0) {
+      tma_prefetch_desc(&P.tmap_B);
+      if (P.rin_tma) tma_prefetch_desc(&P.tmap_R);
+    }
     tmem_alloc(smem_u32(tmem_slot), kExTmemCols);
     tmem_relinquish();
   }
@@ -239,6 +244,15 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
       tma_load_2d(bring + t * P.btile_bytes, &P.tmap_B, bfull0 + 8 * t, 0,
                   static_cast<int>(adapter * n_tot + (c0 - off0)));
     }
+    // Without grouping the piece's rows are contiguous sorted rows: the rank
+    // activations of every slice are one TMA box each (columns j >= r and
+    // rows past the tensor read as zero; rows past the piece feed
+    // accumulator rows that are never stored).
+    if (P.rin_tma) {
+      mbar_arrive_expect_tx(rin_bar, static_cast<uint32_t>(p.S) * P.rin_bytes);
+      for (int q = 0; q < p.S; ++q)
+        tma_load_3d(rin + q * P.rin_bytes, &P.tmap_R, rin_bar, 0, q, pc.lo);
+    }
   }
 
   if (producer) {
@@ -256,10 +270,10 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
       tk = p.permutation ? clampi(__ldg(p.permutation + sr), 0, p.tok - 1) : sr;
     }
     trow[m] = tk;
-    const bool row_ok = m < rows;
+    const bool row_ok = m < rows && !P.rin_tma;
     const uint16_t* src0 = p.in_r + static_cast<int64_t>(sr) * p.ld_in;
     const int nchunk = P.rpad / 8;
-    for (int q = 0; q < p.S; ++q) {
+    for (int q = 0; q < (P.rin_tma ? 0 : p.S); ++q) {
       for (int c = 0; c < nchunk; ++c) {
         const int left = p.r - 8 * c;
         const uint32_t nb = row_ok ? static_cast<uint32_t>(max(0, min(left, 8)) * 2) : 0u;
@@ -327,9 +341,11 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
     // =========================== producers (128 threads)
     // Publish what went out before the barrier, oldest group first: the rank
     // activations (read by the MMA through the async proxy), then each early tile.
-    cp_async_wait_dyn(pre);
-    fence_proxy_async_smem();
-    mbar_arrive(rin_bar);
+    if (!P.rin_tma) {
+      cp_async_wait_dyn(pre);
+      fence_proxy_async_smem();
+      mbar_arrive(rin_bar);
+    }
     for (int t = 0; t < pre; ++t) {
       cp_async_wait_dyn(pre - 1 - t);
       mbar_arrive(xfull0 + 8 * t);

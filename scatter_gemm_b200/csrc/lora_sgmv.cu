@@ -211,6 +211,25 @@ bool encode_2d(CUtensorMap* m, lora_dtype dt, const void* base, uint64_t cols, u
   return r == CUDA_SUCCESS;
 }
 
+// 3-D tiled map: dims {d0 (contiguous), d1, d2}, byte strides s1 (dim 1) and
+// s2 (dim 2), box {b0, b1, b2}.
+bool encode_3d(CUtensorMap* m, lora_dtype dt, const void* base, uint64_t d0, uint64_t d1,
+               uint64_t d2, uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2,
+               CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, dt == LORA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                            : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ workspace
 
 struct Grouping {
@@ -540,6 +559,12 @@ lora_status expand_tc(const lora::ExpandArgs& a, lora_dtype dt, const Grouping& 
   const int64_t n_tot = a.slices.off[a.S] - a.slices.off[0];
   if (!encode_2d(&P.tmap_B, dt, a.B, a.r, static_cast<uint64_t>(a.L) * n_tot,
                  static_cast<uint64_t>(a.rs) * 2, P.rpad, lora::kExBN, swz))
+    return LORA_ERR_CUDA;
+  // the rank activations by TMA when a piece's rows are contiguous sorted rows
+  P.rin_tma = g.row_list == nullptr ? 1 : 0;
+  if (P.rin_tma &&
+      !encode_3d(&P.tmap_R, dt, a.in_r, a.r, a.S, a.tok, static_cast<uint64_t>(a.rs) * 2,
+                 static_cast<uint64_t>(a.ld_in) * 2, P.rpad, 1, lora::kExBM, swz))
     return LORA_ERR_CUDA;
 
   // Tiles per CTA: the split of the tiles into column groups that minimises
