@@ -253,7 +253,7 @@ expand_unaligned_kernel(const __grid_constant__ ExpandUnalignedParams P) {
   // u % 17 (96 = 5 * 17 + 11), so a warp copies two rows' blocks at a time.
   // Eight blocks at a time: their row tokens are read first, then the eight
   // copies issue back to back (a copy may not pass a shared-memory load).
-  auto issue_base = [&](int t, int i, bool publish) {
+  auto issue_base = [&](int t, int i) {
     constexpr int kBaseThreads = 96;
     constexpr int kBatch = 8;
     int q, c0;
@@ -286,7 +286,7 @@ expand_unaligned_kernel(const __grid_constant__ ExpandUnalignedParams P) {
       for (int k = 0; k < kBatch; ++k)
         if (go[k]) cp_async_16(dst[k], src[k], 16u);
     }
-    if (publish) cp_async_arrive_noinc(xfull0 + 8 * (t % NB));
+    cp_async_arrive_noinc(xfull0 + 8 * (t % NB));
     cp_async_commit();
   };
   const int pre = min(NB - 1, ntl);  // base tiles sent at once
@@ -324,7 +324,7 @@ expand_unaligned_kernel(const __grid_constant__ ExpandUnalignedParams P) {
     // whose base area holds staged rank rows until rin_bar).
     cp_async_arrive_noinc(rin_land);
     if (warp != 12)
-      for (int t = 0; t < pre; ++t) issue_base(t, tid - 9 * 32, true);
+      for (int t = 0; t < pre; ++t) issue_base(t, tid - 9 * 32);
     if (warp == 12) {
       // ---- B tiles (warp 12): rows l, l+32, l+64, l+96 of each tile, staged
       //      one tile ahead and realigned; this warp's copies are only its
@@ -369,7 +369,7 @@ expand_unaligned_kernel(const __grid_constant__ ExpandUnalignedParams P) {
         if (t == NB - 1) ok = mbar_wait(rin_bar, 0);
         if (ok && t >= NB) ok = mbar_wait(xempty0 + 8 * s, ((t / NB) - 1) & 1);
         if (!ok) break;
-        issue_base(t, tid - 9 * 32, true);
+        issue_base(t, tid - 9 * 32);
       }
     }
     cp_async_wait<0>();
