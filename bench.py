@@ -652,6 +652,84 @@ def run_e2e(args, probs, lora, device, stream, world):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps}
 
 
+# ----------------------------------------------------------------------------
+# Launch floor: an empty kernel with each of the library's launch shapes
+# ----------------------------------------------------------------------------
+
+# (name, grid, threads, dynamic shared memory bytes, cluster size): the shapes
+# the qkv sweep's kernels launch with (from its ncu launch list)
+LAUNCH_SHAPES = (
+    ("one warp", 1, 32, 0, 1),
+    ("shrink, qkv tok 50", 144, 160, 94408, 16),
+    ("shrink, qkv tok 8192", 288, 160, 94408, 4),
+    ("expand, qkv tok 50", 216, 416, 91784, 1),
+    ("expand, qkv tok 8192", 288, 416, 91784, 1),
+    ("fused, qkv tok 256", 80, 416, 216936, 8),
+)
+
+
+def run_launch_floor(args, device):
+    """Times an empty kernel (compiled here with NVRTC, launched through the
+    driver API) with each launch shape of LAUNCH_SHAPES, with the sweep's
+    method: 256 MB L2-flush write and a GPU sleep before each launch, CUDA
+    events around it.  What remains of a call beyond this is the kernel's own
+    work."""
+    from cuda.bindings import driver as cu, nvrtc
+
+    def check(res):
+        err = res[0]
+        assert int(err) == 0, err
+        return res[1] if len(res) > 1 else None
+
+    prog = check(nvrtc.nvrtcCreateProgram(b'extern "C" __global__ void lora_empty() {}',
+                                          b"empty.cu", 0, [], []))
+    opts = [b"--gpu-architecture=sm_100a"]
+    check(nvrtc.nvrtcCompileProgram(prog, len(opts), opts))
+    cubin = b" " * check(nvrtc.nvrtcGetCUBINSize(prog))
+    check(nvrtc.nvrtcGetCUBIN(prog, cubin))
+    torch.cuda.synchronize()  # the runtime's primary context is current
+    mod = check(cu.cuModuleLoadData(cubin))
+    fn = check(cu.cuModuleGetFunction(mod, b"lora_empty"))
+    fa = cu.CUfunction_attribute
+    check(cu.cuFuncSetAttribute(fn, fa.CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES,
+                                227 * 1024))
+    check(cu.cuFuncSetAttribute(fn, fa.CU_FUNC_ATTRIBUTE_NON_PORTABLE_CLUSTER_SIZE_ALLOWED, 1))
+    stream = torch.cuda.current_stream(device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    nap = 100000
+    rows = []
+    for name, grid, threads, smem, cluster in LAUNCH_SHAPES:
+        cfg = cu.CUlaunchConfig()
+        cfg.gridDimX, cfg.gridDimY, cfg.gridDimZ = grid, 1, 1
+        cfg.blockDimX, cfg.blockDimY, cfg.blockDimZ = threads, 1, 1
+        cfg.sharedMemBytes = smem
+        cfg.hStream = cu.CUstream(stream.cuda_stream)
+        attr = cu.CUlaunchAttribute()
+        attr.id = cu.CUlaunchAttributeID.CU_LAUNCH_ATTRIBUTE_CLUSTER_DIMENSION
+        attr.value.clusterDim.x, attr.value.clusterDim.y, attr.value.clusterDim.z = cluster, 1, 1
+        cfg.attrs = [attr]
+        cfg.numAttrs = 1
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for k in range(args.warmup + args.steps):
+            flush.zero_()
+            torch.cuda._sleep(nap)
+            if k >= args.warmup:
+                ev[k - args.warmup][0].record(stream)
+            check(cu.cuLaunchKernelEx(cfg, fn, None, 0))
+            if k >= args.warmup:
+                ev[k - args.warmup][1].record(stream)
+        torch.cuda.synchronize()
+        t = [a.elapsed_time(b) * 1e3 for a, b in ev]
+        rows.append({"shape": name, "grid": grid, "threads": threads, "smem_bytes": smem,
+                     "cluster": cluster, "us_mean": round(float(np.mean(t)), 2),
+                     "us_median": round(float(np.median(t)), 2)})
+    check(cu.cuModuleUnload(mod))
+    print(json.dumps({"mode": "launch_floor", "unit": "us", "steps": args.steps,
+                      "warmup": args.warmup, "l2": "flushed before every launch (256 MB write), "
+                      "then ~50 us GPU sleep", "launches": rows}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -668,6 +746,8 @@ def main():
     ap.add_argument("--no-configs", action="store_true")
     ap.add_argument("--configs", default="",
                     help="per-config lines to time, e.g. gate_up:fp16,tail:fp16 (default: all)")
+    ap.add_argument("--launch-floor", action="store_true",
+                    help="time an empty kernel with each of the library's launch shapes, then exit")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -682,6 +762,9 @@ def main():
         raise SystemExit("bench.py needs a CUDA device")
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
+    if args.launch_floor:
+        run_launch_floor(args, device)
+        return
     if world > 1:
         import datetime
         import torch.distributed as dist
