@@ -61,6 +61,15 @@ def test_expand_element_aligned_rank64_slice_counts(slices):
         assert lora.last_path() & T
 
 
+def test_expand_element_aligned_rank64_three_slices_grouped():
+    # rank 64, three slices (the last slice's staged rank rows in stage 0, the
+    # first B tile after them) on the grouped schedule
+    p = make_problem("many_small", seed=66, tok=900, nseg=120, K=64, slices=[200, 72, 72],
+                     r=64, rs=64, misalign=1)
+    check_expand(p, workspace=True)
+    assert lora.last_path() & G and lora.last_path() & T
+
+
 def test_expand_element_aligned_grouped_zero_scaling_and_lead_trail():
     p = make_problem("many_small", seed=70, tok=900, nseg=120, K=64, slices=[250, 70, 70],
                      misalign=3, lead=9, trail=4, col_lead=5)
