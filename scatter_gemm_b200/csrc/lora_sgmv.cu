@@ -51,6 +51,9 @@
 #ifndef LORA_EXPAND_B_STAGES
 #define LORA_EXPAND_B_STAGES 3
 #endif
+#ifndef LORA_BASE_EXPAND_CTAS_PER_SM
+#define LORA_BASE_EXPAND_CTAS_PER_SM 2  // base projection: 2 when three stages fit in 113 KB
+#endif
 #ifndef LORA_EU_CTAS_PER_SM
 #define LORA_EU_CTAS_PER_SM 2       // element-aligned expand: CTAs per SM when they fit
 #endif
@@ -1265,7 +1268,7 @@ lora_status base_expand_tc(const lora::BaseExpandArgs& a, const void* W, int64_t
     return static_cast<size_t>(stages) * kStage + P.rin_bytes + P.btile_bytes + 1024 + 512 +
            8 * (2 * stages + 3) + 16;
   };
-  const bool two = total(3) <= 113 * 1024;
+  const bool two = LORA_BASE_EXPAND_CTAS_PER_SM >= 2 && total(3) <= 113 * 1024;
   const size_t cap = (two ? 113 : 225) * 1024;
   P.stages = 2;
   while (P.stages < 6 && total(P.stages + 1) <= cap) ++P.stages;
