@@ -51,6 +51,9 @@
 #ifndef LORA_EXPAND_B_STAGES
 #define LORA_EXPAND_B_STAGES 3
 #endif
+#ifndef LORA_SHRINK_RING_BELOW
+#define LORA_SHRINK_RING_BELOW 3    // split-K partials into the ring below this many stages
+#endif
 #ifndef LORA_BASE_EXPAND_CTAS_PER_SM
 #define LORA_BASE_EXPAND_CTAS_PER_SM 2  // base projection: 2 when three stages fit in 113 KB
 #endif
@@ -438,7 +441,7 @@ lora_status shrink_tc(const lora::ShrinkArgs& a, lora_dtype dt, const Grouping& 
   // the partials are received in the ring, each CTA's once its MMAs are done
   P.stages = stages_for(recv_full);
   P.recv_in_ring = 0;
-  if (cs > 1 && P.stages < 3) {
+  if (cs > 1 && P.stages < LORA_SHRINK_RING_BELOW) {
     P.recv_in_ring = 1;
     P.stages = stages_for(0);
     while (static_cast<size_t>(P.stages) * P.stage_bytes < recv_full) ++P.stages;
