@@ -177,6 +177,10 @@ CONFIGS: Dict[str, Dict] = {
     # 16,384 tokens, one token per segment (the launch-bound regression case)
     "ones16k": dict(dtype="bf16", tok=16384, K=4096, slices=[4096, 1024, 1024],
                     L=8, r=16, rs=16, nseg=16384, recipe="ones", scaling=2.0),
+    # rank 128 on q/k/v slices: beyond the tensor-core kernels' range (rank
+    # <= 64, S*rs <= 256), so both ops run on the CUDA-core kernels
+    "wide_rank": dict(dtype="bf16", tok=1024, K=4096, slices=[4096, 1024, 1024], L=8,
+                      r=128, rs=128, nseg=8, recipe="uniform", scaling=2.0),
 }
 
 QKV_TOK_SWEEP = (50, 128, 256, 512, 1024, 2048, 4096, 6144, 8192)

@@ -132,6 +132,19 @@ def test_grouping_long_segments_and_many_adapters(L, nseg, tok, K):
     assert lora.last_path() & G and lora.last_path() & T
 
 
+# beyond the tensor-core kernels' range (rank > 64; shrink S*rs > 256): the
+# CUDA-core kernels, aligned and at any element offset
+@pytest.mark.parametrize("mis", [0, 1])
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_wide_rank_runs_on_the_cuda_cores(mis, dtype):
+    p = make_problem("wide_rank", seed=27 + mis, tok=300, K=264, slices=[256, 64, 72], r=100,
+                     rs=104, dtype=dtype, misalign=mis, ld_pad=mis, col_lead=mis)
+    check_shrink(p)
+    assert lora.last_path() & GEN
+    check_expand(p)
+    assert lora.last_path() & GEN
+
+
 def test_small_token_counts_split_k_over_a_cluster():
     p = make_problem("qkv", seed=23, tok=50, K=4096)
     check_shrink(p)
