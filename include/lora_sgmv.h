@@ -159,7 +159,9 @@ LORA_API lora_status lora_expand(const void* in_r, int64_t ld_in, const void* B_
                         void* stream);
 
 /* Bytes of optional workspace that lets lora_shrink / lora_expand use the
- * adapter-grouped schedule for tables with many small segments. */
+ * adapter-grouped schedule for tables with many small segments.  The grouping
+ * pass is skipped when it would save under 64 KB of adapter-weight reads
+ * ((nseg - L) times the weights one 128-row piece reads). */
 LORA_API size_t lora_workspace_size(int tok, int nseg, int L);
 
 /* lora_validate -- the value checks of the tables (sgl-kernel-xpu page, section "Behaviour

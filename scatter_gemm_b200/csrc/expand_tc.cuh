@@ -163,6 +163,8 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
     tmem_alloc(smem_u32(tmem_slot), kExTmemCols);
     tmem_relinquish();
   }
+  // the grouping pass ahead of this kernel (when there is one) has finished
+  griddep_wait();
 
   // Producer thread pt owns row pt of the piece.  Rows of a block slot start
   // at slot*128: their sorted rows and tokens are fetched while the tables are read.

@@ -164,6 +164,8 @@ expand_unaligned_kernel(const __grid_constant__ ExpandUnalignedParams P) {
     tmem_alloc(smem_u32(tmem_slot), kExTmemCols);
     tmem_relinquish();
   }
+  // the grouping pass ahead of this kernel (when there is one) has finished
+  griddep_wait();
 
   // a block slot's piece starts at row slot * 128: the producers fetch the
   // tokens of its rows while the tables are read

@@ -18,6 +18,7 @@
 
 #include "common.cuh"
 #include "sched.cuh"
+#include "sm100.cuh"
 
 namespace lora {
 
@@ -55,6 +56,7 @@ group_rows_kernel(const int32_t* __restrict__ seg_indptr, const int32_t* __restr
   extern __shared__ int cnt[];
   __shared__ int warp_tot[32];
   const int tid = threadIdx.x;
+  griddep_launch_dependents();  // the kernel that reads the lists may start its CTAs
   const bool staged = group_stages_tables(nseg, L);
   int* sidx = cnt + L;
   int* swi = sidx + nseg + 1;
@@ -162,6 +164,7 @@ group_rows_small_kernel(const int32_t* __restrict__ seg_indptr,
                         int32_t* __restrict__ vseg_indptr, int32_t* __restrict__ row_list) {
   extern __shared__ int sm[];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  griddep_launch_dependents();  // the kernel that reads the lists may start its CTAs
   constexpr int kWarps = kGroupThreads / 32;
   int* hist = sm;                       // [32][L]: counts, then cursors
   int* sidx = hist + kWarps * L;        // clamped seg_indptr

@@ -244,6 +244,36 @@ struct Grouping {
   int nvseg = 0;
 };
 
+#ifndef LORA_PDL
+#define LORA_PDL 1  // kernels after the grouping pass start while it runs
+#endif
+
+// Launch attributes of a tensor-core kernel: its cluster shape, and, right
+// after the grouping pass, programmatic serialisation: its CTAs are placed and
+// run their set-up (barriers, TMEM) while the pass finishes, then wait for it
+// (griddep_wait) before reading the lists.
+struct LaunchAttrs {
+  cudaLaunchAttribute a[2];
+  unsigned n = 0;
+  void cluster(unsigned x) {
+    a[n].id = cudaLaunchAttributeClusterDimension;
+    a[n].val.clusterDim.x = x;
+    a[n].val.clusterDim.y = 1;
+    a[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  void after_grouping(const Grouping& g) {
+    if (!LORA_PDL || g.vseg_indptr == nullptr) return;
+    a[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  void apply(cudaLaunchConfig_t& cfg) {
+    cfg.attrs = n ? a : nullptr;
+    cfg.numAttrs = n;
+  }
+};
+
 inline size_t a16(size_t n) { return (n + 3) / 4 * 4; }  // ints -> multiple of 4 ints
 
 size_t workspace_ints(int tok, int nseg, int L) {
@@ -314,11 +344,18 @@ lora_status narrow_tables(const int64_t* seg_indptr, const int64_t* weight_indic
 }
 
 // Enqueues the grouping pass when the schedule calls for it.
+// piece_weight_bytes: the adapter weights one piece of rows reads (A for the
+// shrink, B for the expand).  Grouping saves about one such read for every
+// segment beyond one per adapter; below kGroupMinSavedBytes of them the pass
+// (one more kernel on the stream) costs more than it saves.
+constexpr int64_t kGroupMinSavedBytes = 64 * 1024;
+
 lora_status maybe_group(const int32_t* seg_indptr, const int32_t* weight_indices, int tok,
-                        int nseg, int L, void* ws, size_t ws_bytes, cudaStream_t st,
-                        Grouping& g) {
+                        int nseg, int L, int64_t piece_weight_bytes, void* ws, size_t ws_bytes,
+                        cudaStream_t st, Grouping& g) {
   g = Grouping{};
   if (!ws || nseg <= L || L > lora::kGroupMaxAdapters) return LORA_OK;
+  if (static_cast<int64_t>(nseg - L) * piece_weight_bytes < kGroupMinSavedBytes) return LORA_OK;
   if (!device_facts()) return LORA_ERR_CUDA;  // sets the pass's shared-memory limit
   if (!aligned_to(ws, 16) || ws_bytes < workspace_ints(tok, nseg, L) * 4) return LORA_OK;
   int32_t* w = static_cast<int32_t*>(ws);
@@ -451,19 +488,14 @@ lora_status shrink_tc(const lora::ShrinkArgs& a, lora_dtype dt, const Grouping& 
   const size_t smem = smem_need;
   const long slots = lora::num_piece_slots(a.tok, P.nvseg, lora::kTcBM);
   cudaLaunchConfig_t cfg{};
-  cudaLaunchAttribute attr[1];
+  LaunchAttrs attrs;
   cfg.gridDim = dim3(static_cast<unsigned>(slots * cs));
   cfg.blockDim = dim3(lora::kTcThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  if (cs > 1) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-  }
+  if (cs > 1) attrs.cluster(cs);
+  attrs.after_grouping(g);
+  attrs.apply(cfg);
   if (smem > 227 * 1024) return LORA_ERR_UNSUPPORTED;
   cudaError_t e;
   if (!al) e = cudaLaunchKernelEx(&cfg, lora::shrink_tc_kernel<E, 1, false>, P);
@@ -600,6 +632,9 @@ lora_status expand_tc(const lora::ExpandArgs& a, lora_dtype dt, const Grouping& 
   cfg.blockDim = dim3(lora::kExThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
+  LaunchAttrs attrs;
+  attrs.after_grouping(g);
+  attrs.apply(cfg);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, lora::expand_tc_kernel<E>, P);
   ++g_launches;
   g_last_path = LORA_PATH_TENSOR | (P.vseg_indptr ? LORA_PATH_GROUPED : 0);
@@ -689,6 +724,9 @@ lora_status expand_unaligned_tc(const lora::ExpandArgs& a, lora_dtype dt, const 
   cfg.blockDim = dim3(lora::kExThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
+  LaunchAttrs attrs;
+  attrs.after_grouping(g);
+  attrs.apply(cfg);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, lora::expand_unaligned_kernel<E>, P);
   ++g_launches;
   launched = true;
@@ -876,7 +914,8 @@ lora_status lora_shrink(const void* x, int64_t ld_x, const void* A_stack,
   if (shrink_tc_eligible(a)) {
     Grouping g;
     const lora_status gs =
-        maybe_group(seg_indptr, weight_indices, tok, nseg, L, workspace, workspace_bytes, st, g);
+        maybe_group(seg_indptr, weight_indices, tok, nseg, L,
+                    2ll * S * rs * K, workspace, workspace_bytes, st, g);
     if (gs != LORA_OK) return gs;
     return dtype == LORA_BF16 ? shrink_tc<lora::Bf16>(a, dtype, g, *dev, st)
                               : shrink_tc<lora::Fp16>(a, dtype, g, *dev, st);
@@ -914,7 +953,8 @@ lora_status lora_expand(const void* in_r, int64_t ld_in, const void* B_stack,
   if (expand_tc_eligible(a)) {
     Grouping g;
     const lora_status gs =
-        maybe_group(seg_indptr, weight_indices, tok, nseg, L, workspace, workspace_bytes, st, g);
+        maybe_group(seg_indptr, weight_indices, tok, nseg, L,
+                    2ll * rs * (tab.off[S] - tab.off[0]), workspace, workspace_bytes, st, g);
     if (gs != LORA_OK) return gs;
     return dtype == LORA_BF16 ? expand_tc<lora::Bf16>(a, dtype, g, *dev, st)
                               : expand_tc<lora::Fp16>(a, dtype, g, *dev, st);
@@ -922,7 +962,8 @@ lora_status lora_expand(const void* in_r, int64_t ld_in, const void* B_stack,
   {
     Grouping g;
     const lora_status gs =
-        maybe_group(seg_indptr, weight_indices, tok, nseg, L, workspace, workspace_bytes, st, g);
+        maybe_group(seg_indptr, weight_indices, tok, nseg, L,
+                    2ll * rs * (tab.off[S] - tab.off[0]), workspace, workspace_bytes, st, g);
     if (gs != LORA_OK) return gs;
     bool launched = false;
     const lora_status us = dtype == LORA_BF16

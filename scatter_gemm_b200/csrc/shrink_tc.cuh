@@ -141,6 +141,10 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
   const bool early_arrive = P.csplit > 1;
   if (early_arrive) cluster_arrive_relaxed();
 
+  // the grouping pass ahead of this kernel (when there is one) has finished:
+  // everything above overlapped it
+  griddep_wait();
+
   // ---- piece of this cluster (identical in all its CTAs).  Rows of a block
   // slot start at slot*128, so their tokens are fetched while the tables are read.
   const bool block_slot = slot < (p.tok + kTcBM - 1) / kTcBM;
