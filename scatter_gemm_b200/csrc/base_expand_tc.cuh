@@ -320,7 +320,7 @@ base_expand_tc_kernel(const __grid_constant__ BaseExpandTcParams P) {
           const int row = u / 16, c = u % 16;
           const int col = c0 + 8 * c;
           if (row < rows && col < cend)
-            *reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(tk[k]) * p.ld_out + col) = w[k];
+            stg128(p.out + static_cast<int64_t>(tk[k]) * p.ld_out + col, w[k]);
         }
       }
     }

@@ -65,6 +65,29 @@ struct SliceTable {
   int S;
 };
 
+// Stores to global memory by explicit global-space instructions.  A store
+// through a generic pointer might alias shared memory, so shared-memory loads
+// issued after it wait behind it; these stores cannot alias it.
+__device__ __forceinline__ void stg128(void* p, uint4 v) {
+  asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(__cvta_generic_to_global(p)),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ void stg64(void* p, uint2 v) {
+  asm volatile("st.global.v2.b32 [%0], {%1, %2};" ::"l"(__cvta_generic_to_global(p)), "r"(v.x),
+               "r"(v.y)
+               : "memory");
+}
+
+__device__ __forceinline__ void stg32(void* p, uint32_t v) {
+  asm volatile("st.global.b32 [%0], %1;" ::"l"(__cvta_generic_to_global(p)), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void stg16(void* p, uint16_t v) {
+  asm volatile("st.global.b16 [%0], %1;" ::"l"(__cvta_generic_to_global(p)), "h"(v) : "memory");
+}
+
 // Column c (global base-output column) -> its slice q.
 __device__ __forceinline__ int slice_of(const SliceTable& st, int c) {
   int q = 0;

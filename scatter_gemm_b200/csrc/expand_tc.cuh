@@ -437,8 +437,7 @@ expand_tc_kernel(const __grid_constant__ ExpandTcParams P) {
           const int row = u / kExCh, c = u % kExCh;
           const int col = c0 + 8 * c;
           if (row < rows && col < cend)
-            *reinterpret_cast<uint4*>(p.base + static_cast<int64_t>(tk[j]) * p.ld_base + col) =
-                w[j];
+            stg128(p.base + static_cast<int64_t>(tk[j]) * p.ld_base + col, w[j]);
         }
       }
       mbar_arrive(xempty0 + 8 * s);  // the stage's shared memory may be refilled

@@ -494,13 +494,13 @@ expand_unaligned_kernel(const __grid_constant__ ExpandUnalignedParams P) {
               const uint8_t* src = rowp + 16 * b + 2 * i;
               uint8_t* dst = reinterpret_cast<uint8_t*>(ga) + 2 * i;
               if ((i & 3) == 0 && i + 4 <= i1) {
-                *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(src);
+                stg64(dst, *reinterpret_cast<const uint2*>(src));
                 i += 4;
               } else if ((i & 1) == 0 && i + 2 <= i1) {
-                *reinterpret_cast<uint32_t*>(dst) = *reinterpret_cast<const uint32_t*>(src);
+                stg32(dst, *reinterpret_cast<const uint32_t*>(src));
                 i += 2;
               } else {
-                *reinterpret_cast<uint16_t*>(dst) = *reinterpret_cast<const uint16_t*>(src);
+                stg16(dst, *reinterpret_cast<const uint16_t*>(src));
                 i += 1;
               }
             }
@@ -513,7 +513,7 @@ expand_unaligned_kernel(const __grid_constant__ ExpandUnalignedParams P) {
       // (b) write-back of the whole blocks on the rows' own 16-byte grid:
       //     block u = gt + 128 j -> row u / 17, block u % 17 (128 = 7 * 17 + 9)
       //     Four blocks at a time: every shared-memory load first, then the
-      //     four stores (a load may not pass a store through a generic pointer).
+      //     four stores (global-space stores: the next loads need not wait on them).
       if (ok) {
         constexpr int kBatch = 4;
         int row = gt / kEuRawBlocks, b = gt - row * kEuRawBlocks;
@@ -537,7 +537,7 @@ expand_unaligned_kernel(const __grid_constant__ ExpandUnalignedParams P) {
           }
 #pragma unroll
           for (int k = 0; k < kBatch; ++k)
-            if (go[k]) *reinterpret_cast<uint4*>(ga[k]) = val[k];
+            if (go[k]) stg128(reinterpret_cast<void*>(ga[k]), val[k]);
         }
       }
       group_sync(grp);  // the stage may be refilled

@@ -376,7 +376,7 @@ fused_tc_kernel(const __grid_constant__ FusedTcParams P) {
         uint16_t* orow = ps.out + static_cast<int64_t>(pc.lo + row) * ps.ld_out;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          if (j + k < ps.r) orow[n + k] = b[k];
+          if (j + k < ps.r) stg16(orow + n + k, b[k]);
       }
       // the rounded activations into every CTA's buffer, in the expand's layout
       const uint32_t dst = rin + q * P.rin_bytes + row * (P.rpad * 2) +
@@ -487,7 +487,7 @@ fused_tc_kernel(const __grid_constant__ FusedTcParams P) {
       // (b) coalesced write-back of the rows of the piece: chunk u = j*128 + gt
       const int cend = pe.slices.off[q + 1];
       //     four chunks at a time: their shared-memory reads first, then the
-      //     stores (a load may not pass a store through a generic pointer)
+      //     stores (global-space stores: the next loads need not wait on them)
       if (ok) {
         constexpr int kPer = (kExBM * kExCh) / kFuGroup;
         constexpr int kBatch = 4;
@@ -509,8 +509,7 @@ fused_tc_kernel(const __grid_constant__ FusedTcParams P) {
             const int row = u / kExCh, c = u % kExCh;
             const int col = c0 + 8 * c;
             if (row < rows && col < cend)
-              *reinterpret_cast<uint4*>(pe.base + static_cast<int64_t>(tk[k]) * pe.ld_base + col) =
-                  w[k];
+              stg128(pe.base + static_cast<int64_t>(tk[k]) * pe.ld_base + col, w[k]);
           }
         }
       }

@@ -435,12 +435,12 @@ shrink_tc_kernel(const __grid_constant__ ShrinkTcParams P) {
       w.y = E::f2_to_u32(v[2], v[3]);
       w.z = E::f2_to_u32(v[4], v[5]);
       w.w = E::f2_to_u32(v[6], v[7]);
-      *reinterpret_cast<uint4*>(orow + n0) = w;
+      stg128(orow + n0, w);
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int n = n0 + i;
-        if (n < nvalid && (n % p.rs) < p.r) orow[n] = E::f32_to_bits(v[i]);
+        if (n < nvalid && (n % p.rs) < p.r) stg16(orow + n, E::f32_to_bits(v[i]));
       }
     }
   };
