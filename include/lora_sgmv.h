@@ -249,11 +249,13 @@ LORA_API lora_status lora_embedding_a(const int32_t* ids, const void* A_emb,
  * (1 MiB) compiled into the library, which every GPU that loads the library
  * holds until the process exits.
  *
- *  - Limit: only calls with more segments than adapters (nseg > L) use the
- *    scratch.  For them lora_workspace_size(tok, nseg, L) must not exceed
- *    LORA_STATIC_SCRATCH_BYTES (about tok + nseg + L <= 262,000); larger
- *    problems return LORA_ERR_UNSUPPORTED before anything is enqueued.  Calls
- *    with nseg <= L need no scratch and have no such limit.
+ *  - Limit: only calls that group use the scratch: more segments than
+ *    adapters (nseg > L), and at least 64 KB of weight reads saved
+ *    ((nseg - L) * S * rs * K * 2 bytes).  For them lora_workspace_size(tok,
+ *    nseg, L) must not exceed LORA_STATIC_SCRATCH_BYTES (about
+ *    tok + nseg + L <= 262,000); larger problems return LORA_ERR_UNSUPPORTED
+ *    before anything is enqueued.  Other calls need no scratch and have no
+ *    such limit.
  *  - The first call on each device looks up the array's device address with
  *    that device current (a CUDA runtime query, no allocation) and caches it;
  *    make that first call before any stream capture.  The cached address

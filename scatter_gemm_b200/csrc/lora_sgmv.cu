@@ -350,12 +350,16 @@ lora_status narrow_tables(const int64_t* seg_indptr, const int64_t* weight_indic
 // (one more kernel on the stream) costs more than it saves.
 constexpr int64_t kGroupMinSavedBytes = 64 * 1024;
 
+bool grouping_pays(int nseg, int L, int64_t piece_weight_bytes) {
+  return nseg > L && L <= lora::kGroupMaxAdapters &&
+         static_cast<int64_t>(nseg - L) * piece_weight_bytes >= kGroupMinSavedBytes;
+}
+
 lora_status maybe_group(const int32_t* seg_indptr, const int32_t* weight_indices, int tok,
                         int nseg, int L, int64_t piece_weight_bytes, void* ws, size_t ws_bytes,
                         cudaStream_t st, Grouping& g) {
   g = Grouping{};
-  if (!ws || nseg <= L || L > lora::kGroupMaxAdapters) return LORA_OK;
-  if (static_cast<int64_t>(nseg - L) * piece_weight_bytes < kGroupMinSavedBytes) return LORA_OK;
+  if (!ws || !grouping_pays(nseg, L, piece_weight_bytes)) return LORA_OK;
   if (!device_facts()) return LORA_ERR_CUDA;  // sets the pass's shared-memory limit
   if (!aligned_to(ws, 16) || ws_bytes < workspace_ints(tok, nseg, L) * 4) return LORA_OK;
   int32_t* w = static_cast<int32_t*>(ws);
@@ -1135,8 +1139,9 @@ extern "C" lora_status lora_shrink_static_scratch(
     const int32_t* weight_indices, const int32_t* permutation, void* out_r, int64_t ld_out,
     int tok, int K, int S, int r, int rs, int nseg, int L, lora_dtype dtype, void* stream) {
   // Only the adapter-grouping pass uses scratch, and it runs only with more
-  // segments than adapters; any other call needs none, so it has no size limit.
-  if (!(nseg > L && L <= lora::kGroupMaxAdapters))
+  // segments than adapters and enough weight reads to save; any other call
+  // needs none, so it has no size limit.
+  if (!grouping_pays(nseg, L, 2ll * S * rs * K))
     return lora_shrink(x, ld_x, A_stack, seg_indptr, weight_indices, permutation, out_r,
                        ld_out, tok, K, S, r, rs, nseg, L, dtype, nullptr, 0, stream);
   // the grouping pass writes every word of the scratch it later reads, so

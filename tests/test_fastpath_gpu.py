@@ -116,6 +116,18 @@ def test_many_segments_with_workspace_are_grouped():
     assert not lora.last_path() & G
 
 
+def test_grouping_skipped_when_it_saves_little():
+    # 3 segments of 2 adapters, K = 512, rank 8: one extra piece saves 8 KB of
+    # weight reads, under the grouping pass's 64 KB threshold, so a workspace
+    # is left unused and the result is still the oracle's
+    p = make_problem("tiny", seed=77)
+    assert p.nseg > p.L
+    check_shrink(p, workspace=True)
+    assert lora.last_path() & T and not lora.last_path() & G
+    check_expand(p, workspace=True)
+    assert lora.last_path() & T and not lora.last_path() & G
+
+
 @pytest.mark.parametrize("L,nseg,tok,K", [(8, 20, 2000, 192), (300, 400, 1200, 192),
                                            (16, 2100, 30000, 64)])
 def test_grouping_long_segments_and_many_adapters(L, nseg, tok, K):

@@ -100,16 +100,21 @@ def test_static_scratch_refuses_problems_beyond_its_size():
     assert st == lora.LORA_ERR_UNSUPPORTED
 
 
-def test_static_scratch_without_grouping_has_no_size_limit():
-    # no more segments than adapters: the call needs no scratch, so a token
-    # count whose grouping workspace would exceed the array still runs
+@pytest.mark.parametrize("nseg", [4, 8])
+def test_static_scratch_without_grouping_has_no_size_limit(nseg):
+    # no grouping, so no scratch: either no more segments than adapters, or
+    # 8 segments of 4 adapters whose pieces read 1 KB of weights each (4 KB
+    # saved, under the pass's 64 KB threshold); a token count whose grouping
+    # workspace would exceed the array still runs
     tok, K, S, rs, L = 270_000, 64, 1, 8, 4
-    assert lora.workspace_size(tok, L, L) > lora.STATIC_SCRATCH_BYTES
+    assert lora.workspace_size(tok, nseg, L) > lora.STATIC_SCRATCH_BYTES
     g = torch.Generator(device="cuda").manual_seed(5)
     x = torch.randn(tok, K, device="cuda", generator=g).to(torch.bfloat16)
     A = (0.02 * torch.randn(L, S * rs, K, device="cuda", generator=g)).to(torch.bfloat16)
-    si = torch.tensor([0, 60_000, 130_000, 200_000, tok], dtype=torch.int32, device="cuda")
-    wi = torch.tensor([2, 0, 3, 1], dtype=torch.int32, device="cuda")
+    bounds = [0, 60_000, 130_000, 200_000, tok] if nseg == 4 else \
+        [0, 30_000, 60_000, 95_000, 130_000, 165_000, 200_000, 235_000, tok]
+    si = torch.tensor(bounds, dtype=torch.int32, device="cuda")
+    wi = torch.tensor([2, 0, 3, 1, 2, 0, 3, 1][:nseg], dtype=torch.int32, device="cuda")
     pm = torch.randperm(tok, device="cuda", generator=g).to(torch.int32)
     ref = torch.zeros(tok, S * rs, dtype=torch.bfloat16, device="cuda")
     lora.lora_shrink(x, A, si, wi, pm, ref, num_slices=S)
