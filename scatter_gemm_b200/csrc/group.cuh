@@ -3,11 +3,14 @@
 // The sgl-kernel-xpu page ("Decode LoRA kernels are optimized", section
 // "Behaviour changes") asks callers to pass one coalesced segment per adapter
 // because the kernels tile M themselves.  When a caller does not (here: more
-// segments than adapters and a workspace to work in), this single-CTA pass
-// coalesces on the device instead: it lists the rows of every adapter's
-// segments contiguously, so the tensor-core kernels tile each adapter's rows
-// in 128-row pieces and read each adapter's weights once per piece instead of
-// once per segment.  Nothing is synchronised with the host.
+// segments than adapters, at least 64 KB of weight reads to save, and a
+// workspace to work in), this single-CTA pass coalesces on the device
+// instead: it lists the rows of every adapter's segments contiguously, so the
+// tensor-core kernels tile each adapter's rows in 128-row pieces and read each
+// adapter's weights once per piece instead of once per segment.  Nothing is
+// synchronised with the host; the kernel after the pass may start its CTAs
+// while the pass runs (programmatic dependent launch) and waits for it before
+// reading the lists.
 //
 // Workspace layout (int32): vseg_indptr[L+1] | seg_base[nseg] | row_list[tok]
 //   vseg_indptr  rows of adapter a are grouped rows [vseg_indptr[a], vseg_indptr[a+1])

@@ -11,8 +11,9 @@
 //   tensor it streams is 16-byte aligned with 16-byte-multiple row strides,
 //   slice starts % 8 == 0 and r <= 64, else expand_unaligned for r <= 64; the
 //   CUDA-core kernels of general.cuh for what remains (r > 64, S*rs > 256).
-//   With a workspace and more segments than adapters the tensor-core kernels
-//   run on the adapter-grouped schedule of group.cuh.
+//   With a workspace, more segments than adapters and at least 64 KB of
+//   weight reads to save, the tensor-core kernels run on the adapter-grouped
+//   schedule of group.cuh.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
