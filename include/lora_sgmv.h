@@ -52,7 +52,10 @@
  *    error code (lora_device_error) and lets the kernel finish without
  *    writing further results.  Thread-block-cluster barriers and the TMEM
  *    allocation are not bounded this way; the rule above keeps them from
- *    waiting on anything but the cluster's own thread blocks.
+ *    waiting on anything but the cluster's own thread blocks.  A kernel that
+ *    follows the adapter-grouping pass may start before the pass ends and
+ *    then waits for it (programmatic dependent launch); the pass is one
+ *    thread block with no waits of its own.
  *  - Invalid table VALUES (a decreasing seg_indptr, an adapter index out of
  *    range, a permutation that is not a bijection) are undefined behaviour in
  *    lora_shrink / lora_expand, as on the pages (section "Behaviour changes");
@@ -360,9 +363,10 @@ LORA_API lora_status lora_expand_i64(const void* in_r, int64_t ld_in, const void
  * call made on this host thread; 0 if none launched a kernel. */
 LORA_API int lora_last_path(void);
 
-/* Failure detection of the tensor-core kernels.  Every wait inside them is
- * bounded (1 s); a wait that runs out records a nonzero code in a device word,
- * and the kernel releases its resources and returns without further writes.
+/* Failure detection of the tensor-core kernels.  Every mbarrier wait inside
+ * them is bounded (1 s); a wait that runs out records a nonzero code in a
+ * device word, and the kernel releases its resources and returns without
+ * further writes.
  * This call reads that word (synchronously, on the current device) into *code
  * and clears it if `clear` is nonzero. */
 LORA_API lora_status lora_device_error(int32_t* code, int clear);
